@@ -1,0 +1,289 @@
+/*
+ * tree_verify.h -- C ABI of the tree-verification library (libtreeverify.so).
+ *
+ * One speculative-decoding iteration verifies a whole draft token tree
+ * against the target model in one pass (SpecExec: Massively Parallel
+ * Speculative Decoding For Interactive LLM Inference on Consumer Devices,
+ * "Approach").  This library implements the data-parallel hot path of that
+ * step as three calls, each a set of hand-written CUDA kernels for sm_100a:
+ *
+ *   tree_verify_attn  -- tree-masked attention of every draft node over the
+ *                        shared KV-cache prefix plus its own ancestors
+ *                        (EasySpec page, "Experimental setup", the "+tree"
+ *                        baseline; SpecExec page, "Approach"), optionally
+ *                        restricted to the top-k prefix blocks chosen by a
+ *                        cheap block-mean score ("Accelerate Speculative
+ *                        Decoding with Sparse Computation in Verification",
+ *                        "Methodology" 3, attention sparsity);
+ *   tree_accept       -- the acceptance walk over the verified tree: greedy
+ *                        longest match at temperature 0, multi-draft
+ *                        speculative sampling with residual resampling
+ *                        (SpecExec page, "Builds on": speculative sampling,
+ *                        SpecInfer), or SpecExec's sample-and-descend rule
+ *                        for deterministic trees (SpecExec page, "Approach");
+ *   tree_expand_topb  -- one round of SpecExec's batched best-first
+ *                        (Dijkstra-style) tree construction that keeps the
+ *                        highest cumulative-probability continuations
+ *                        (SpecExec page, "Approach"; "Builds on": Dijkstra's
+ *                        algorithm).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every array pointer is DEVICE memory owned by the caller, unless the
+ *   field says otherwise.  The argument structs themselves live in host
+ *   memory and are read during the call only.
+ * - Calls enqueue work on the caller's stream and never synchronise.  They
+ *   return a tv_status after host-side argument checks and the launches
+ *   (cudaGetLastError); a TV_OK return does not mean the kernels finished.
+ * - The library keeps no state between calls and allocates nothing; scratch
+ *   comes from a caller buffer `ws` of at least *_workspace_size() bytes
+ *   (256-byte aligned).  The workspace must be zero-filled once before its
+ *   first use; every call leaves it ready for the next one.  Two calls that
+ *   may run concurrently must not share a workspace.
+ * - Data-dependent faults are never trapped: the kernels OR bits into the
+ *   caller's `dev_status` word (a device uint32, may be NULL) and write the
+ *   documented defined output (NaN or -1) instead.
+ * - A draft tree is a parent[] array: node 0 is the root (the last committed
+ *   token), parent[0] = -1 and 0 <= parent[i] < i (topological order).  A
+ *   node attends to itself; the root's row predicts the first new token.
+ * - Tree node counts n_nodes[b] <= T may be given per sequence (device
+ *   int32 array) or NULL (= T for every sequence).
+ */
+#ifndef TREE_VERIFY_H
+#define TREE_VERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TV_API __attribute__((visibility("default")))
+#else
+#define TV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (cudaStream_t); NULL is the legacy default stream. */
+typedef struct CUstream_st* tv_stream_t;
+
+/* Host-side result of a call. */
+typedef enum {
+  TV_OK = 0,
+  TV_ERR_INVALID_ARG = 1,   /* a host-checkable argument is out of range  */
+  TV_ERR_UNSUPPORTED = 2,   /* valid, but outside what the kernels handle */
+  TV_ERR_WORKSPACE = 3,     /* ws is NULL, misaligned or too small        */
+  TV_ERR_CUDA = 4           /* a CUDA launch or API call failed           */
+} tv_status;
+
+/* Device status bits (ORed into *dev_status by the kernels). */
+enum {
+  TV_DEV_BAD_PARENT = 1,    /* parent[0] != -1 or parent[i] not in [0, i)  */
+  TV_DEV_BAD_TOKEN = 2,     /* a draft token outside [0, V)                */
+  TV_DEV_NONFINITE = 4,     /* NaN/Inf logits, or invalid probabilities    */
+  TV_DEV_BAD_ROW = 8,       /* expansion row for a missing/expanded node   */
+  TV_DEV_BAD_LEN = 16       /* n_nodes or prefix_len out of range          */
+};
+
+typedef enum { TV_FP32 = 0, TV_BF16 = 1 } tv_dtype;
+
+/* ------------------------------------------------------------------------
+ * tree_verify_attn
+ *
+ * For sequence b, draft node i < n_nodes[b] and query head h (kv head
+ * g = h / (Hq / Hkv), contiguous GQA groups), with K(i) = prefix positions
+ * 0 .. prefix_len[b]-1 of the cache plus the tree nodes on the path
+ * root .. i (i included):
+ *     out[b][i][h] = sum_{j in K(i)} softmax_j(scale * <q, k_j>) v_j
+ *     lse[b][i][h] = log sum_{j in K(i)} exp(scale * <q, k_j>)   (natural log)
+ * Queries and keys arrive post-RoPE; the caller positions node i at
+ * prefix_len[b] + depth(i).  scale = 0 means 1/sqrt(d).
+ *
+ * Block top-k (sparse_topk > 0): the prefix is cut into blocks of
+ * block_size positions; kbar[b][j][g] is the mean of block j's valid keys;
+ * for each (b, i, g) the sparse_topk blocks with the largest
+ * sum_{h in group g} <q_{i,h}, kbar_j> (ties: lower block index) are kept
+ * and K(i) = their keys plus the tree path.  With at most sparse_topk
+ * blocks every block is kept (identical to dense).
+ *
+ * Layouts (element strides; the innermost dimension d is contiguous):
+ *   q        [B][T][Hq][d]      strides q_sb, q_st, q_sh
+ *   k_cache, v_cache  [B][Lmax][Hkv][d]  strides kv_sb, kv_sl, kv_sh (shared)
+ *   k_tree, v_tree    [B][T][Hkv][d]     strides kt_sb, kt_st, kt_sh (shared)
+ *   out      [B][T][Hq][d]      strides o_sb, o_st, o_sh   (dtype of q)
+ *   lse      [B][T][Hq] fp32 contiguous, or NULL
+ *   parent   [B][T] int32, row stride parent_sb
+ *   prefix_len [B] int32 (device), each in [0, Lmax]
+ *   k_block_mean [B][ceil(Lmax/block_size)][Hkv][d] fp32 contiguous, or NULL
+ *            (then computed inside the call)
+ *   sel_blocks   [B][T][Hkv][sparse_topk] int32 or NULL: kept block ids,
+ *            ascending, -1 padded
+ * dtype: TV_FP32 (d in {32, 64, 128}) or TV_BF16 (d in {64, 128}); all of
+ * q, caches, tree K/V and out share it.  B, T, Hq, Hkv >= 0; Hq % Hkv == 0.
+ * Rows i >= n_nodes[b] are not written.  A node whose parent chain is
+ * malformed gets NaN rows (TV_DEV_BAD_PARENT); a sequence whose prefix_len
+ * is outside [0, Lmax] gets NaN rows and one whose n_nodes is outside
+ * [0, T] gets none (TV_DEV_BAD_LEN).
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int32_t dtype;
+  int32_t B, T, Hq, Hkv, d, Lmax;
+  const void* q;        int64_t q_sb, q_st, q_sh;
+  const void* k_cache;
+  const void* v_cache;  int64_t kv_sb, kv_sl, kv_sh;
+  const int32_t* prefix_len;
+  const void* k_tree;
+  const void* v_tree;   int64_t kt_sb, kt_st, kt_sh;
+  const int32_t* parent; int64_t parent_sb;
+  const int32_t* n_nodes;
+  float scale;
+  int32_t sparse_topk;
+  int32_t block_size;
+  const float* k_block_mean;
+  void* out;            int64_t o_sb, o_st, o_sh;
+  float* lse;
+  int32_t* sel_blocks;
+  uint32_t* dev_status;
+} tv_attn_args;
+
+TV_API size_t tree_verify_attn_workspace_size(const tv_attn_args* a);
+TV_API tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws_bytes,
+                           tv_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * tree_accept
+ *
+ * Walks each sequence's tree from the root.  Row c of target_logits is the
+ * target's logits after node c; row c of draft_probs is the draft
+ * distribution node c's children were drawn from.  Children are tried in
+ * ascending node index.
+ *   GREEDY      a = argmax z_c (lowest index on ties); descend to the
+ *               lowest-index child carrying a, else emit a and stop.
+ *   SPECSAMPLE  p = softmax(z_c / temperature); child j (token x_j) is
+ *               accepted when u_j < p(x_j) / q_c(x_j); on rejection p
+ *               becomes (p - q_c)^+ / sum (p - q_c)^+ (unchanged when that
+ *               sum is 0); with every child rejected (or at a leaf) emit
+ *               the inverse-CDF sample of p (smallest t with
+ *               sum_{s<=t} p_s > u * sum p) and stop.
+ *   SPECEXEC    x = inverse-CDF sample of softmax(z_c / temperature);
+ *               descend to the lowest-index child carrying x, else emit x.
+ *   AUTO        GREEDY at temperature 0, else SPECSAMPLE.
+ * temperature 0 means GREEDY in every mode.  Uniforms: Philox4x32-10
+ * (Salmon et al., SC'11) with key (seed mod 2^32, seed >> 32) and counter
+ * (node, b, (tag << 28) | draw, step mod 2^32); u = top 53 bits of
+ * (w0 << 32 | w1) times 2^-53; tag 1 = test of the node's child number
+ * `draw`, tag 2 = residual sample, tag 3 = deterministic-tree sample.
+ *
+ * Inputs:  target_logits [B][T][V] fp32 (row strides tl_sb, tl_st, rows
+ *          contiguous); draft_probs [B][T][V] fp32 (dp_sb, dp_st), required
+ *          for SPECSAMPLE at temperature > 0, else may be NULL;
+ *          draft_tokens [B][T] int32 (tok_sb; entry 0 is ignored);
+ *          parent [B][T] int32 (parent_sb); n_nodes [B] or NULL.
+ * Outputs: n_accepted [B]; accepted_nodes [B][T] (the accepted path without
+ *          the root, -1 padded); out_tokens [B][T+1] (accepted draft tokens
+ *          then the bonus token, -1 padded); min_margin [B] fp64 or NULL
+ *          (smallest |u - ratio| or relative inverse-CDF margin met on the
+ *          path; +inf when none) -- all contiguous.
+ * Faults: children with tokens outside [0, V) are skipped (TV_DEV_BAD_TOKEN);
+ *          nodes with a malformed parent are nobody's child
+ *          (TV_DEV_BAD_PARENT); a visited non-finite row stops the walk with
+ *          bonus -1 (TV_DEV_NONFINITE); n_nodes outside [0, T] accepts
+ *          nothing (TV_DEV_BAD_LEN).
+ * ---------------------------------------------------------------------- */
+typedef enum {
+  TV_ACCEPT_AUTO = 0,
+  TV_ACCEPT_GREEDY = 1,
+  TV_ACCEPT_SPECSAMPLE = 2,
+  TV_ACCEPT_SPECEXEC = 3
+} tv_accept_mode;
+
+typedef struct {
+  int32_t B, T, V;
+  const float* target_logits;  int64_t tl_sb, tl_st;
+  const float* draft_probs;    int64_t dp_sb, dp_st;
+  const int32_t* draft_tokens; int64_t tok_sb;
+  const int32_t* parent;       int64_t parent_sb;
+  const int32_t* n_nodes;
+  int32_t mode;
+  float temperature;
+  uint64_t seed;
+  uint64_t step;
+  int32_t* n_accepted;
+  int32_t* accepted_nodes;
+  int32_t* out_tokens;
+  double* min_margin;
+  uint32_t* dev_status;
+} tv_accept_args;
+
+TV_API size_t tree_accept_workspace_size(const tv_accept_args* a);
+TV_API tv_status tree_accept(const tv_accept_args* a, void* ws, size_t ws_bytes,
+                      tv_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * tree_expand_topb
+ *
+ * One round of batched best-first expansion.  Tree state (caller-owned
+ * device memory, persistent across rounds, set up by tree_expand_init):
+ *   n_nodes [1] int32, parent/token [budget] int32, logp [budget] fp64
+ *   (cumulative draft log-probability; root 0), and an opaque candidate
+ *   pool of tree_expand_pool_bytes(budget, V) bytes.
+ * Per call: R rows of draft logits draft_logits [R][V] fp32 (row stride
+ * ld_logits elements), row r holding the draft logits after tree node
+ * row_node[r] (-1 = no row).  Every (node, token) becomes a candidate with
+ *     score = (logp[node] + z[token] / draft_temperature) - lse(node)
+ * (lse = logsumexp of z / draft_temperature over the row, fp64); the call
+ * appends the sel = min(Bsel, budget - n_nodes) best candidates of the pool
+ * plus the new rows under the total order (score desc, parent asc, token
+ * asc) as nodes n_nodes, n_nodes+1, ... in that order, writes them to
+ * frontier [Bsel] (-1 padded) and *n_appended, and keeps the rest of the
+ * candidates that can still be taken in the pool.  A row for a node that
+ * is not yet in the tree or was expanded before is skipped
+ * (TV_DEV_BAD_ROW); a row with a non-finite logit is skipped
+ * (TV_DEV_NONFINITE).
+ * Limits: 1 <= budget <= 8192, 1 <= V <= 262144, 1 <= Bsel,
+ * draft_temperature > 0.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int32_t V, R, Bsel, budget;
+  float draft_temperature;
+  const float* draft_logits;  int64_t ld_logits;
+  const int32_t* row_node;
+  int32_t* n_nodes;
+  int32_t* parent;
+  int32_t* token;
+  double* logp;
+  void* pool;                 size_t pool_bytes;
+  int32_t* frontier;
+  int32_t* n_appended;
+  uint32_t* dev_status;
+} tv_expand_args;
+
+TV_API size_t tree_expand_pool_bytes(int32_t budget, int32_t V);
+TV_API size_t tree_expand_workspace_size(const tv_expand_args* a);
+/* Resets the tree to the root alone (token root_token, logp 0) and empties
+ * the pool.  The pool needs no other initialisation. */
+TV_API tv_status tree_expand_init(const tv_expand_args* a, int32_t root_token,
+                           tv_stream_t stream);
+TV_API tv_status tree_expand_topb(const tv_expand_args* a, void* ws, size_t ws_bytes,
+                           tv_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Utilities
+ * ---------------------------------------------------------------------- */
+/* Library version, e.g. "treeverify 0.1.0 sm_100a". */
+TV_API const char* tree_verify_version(void);
+/* Static text for a tv_status value. */
+TV_API const char* tv_status_string(tv_status s);
+/* The acceptance uniforms of n draws, computed by the device Philox used in
+ * tree_accept: out[k] = u(seed, step, b[k], node[k], draw[k], tag[k]).
+ * All arrays are device memory of n entries. */
+TV_API tv_status tv_philox_uniforms(uint64_t seed, uint64_t step, const int32_t* b,
+                             const int32_t* node, const int32_t* draw,
+                             const int32_t* tag, double* out, int32_t n,
+                             tv_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TREE_VERIFY_H */

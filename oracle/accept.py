@@ -118,7 +118,7 @@ def tree_accept(target_logits, draft_probs, draft_tokens, parent, n_nodes=None,
     tok = _i64(draft_tokens)
     par = _i64(parent)
     nn = _i64(n_nodes) if n_nodes is not None else np.full(B, T, dtype=np.int64)
-    tau = float(temperature)
+    tau = float(np.float32(temperature))     # the call takes an fp32 temperature
     if tau <= 0.0:
         mode = GREEDY
     elif mode == AUTO:

@@ -32,7 +32,7 @@ The budget counts the root.
 
 Status bits: BAD_ROW (8) for a row whose node is not in the tree or was
 already expanded (the row is skipped); NONFINITE (4) for a row holding a
-non-finite logit (skipped).
+non-finite logit (skipped; the node still counts as expanded).
 """
 
 from __future__ import annotations
@@ -63,7 +63,7 @@ class ExpandState:
 
 def row_scores(logp_n: float, z, tau: float):
     """Cumulative log-probabilities of the V children of one node."""
-    x = _f64(z) / float(tau)
+    x = _f64(z) / float(np.float32(tau))     # the call takes an fp32 temperature
     m = np.max(x)
     lse = m + np.log(np.sum(np.exp(x - m)))
     return (logp_n + x) - lse
@@ -84,11 +84,11 @@ def expand_call(st: ExpandState, draft_logits, row_node, Bsel: int, tau: float =
         if n >= st.n_nodes or n in st.expanded:
             st.status |= ST_BAD_ROW
             continue
+        st.expanded.add(n)                      # a row is consumed once given
         z = _f64(Zd[r])
         if not np.all(np.isfinite(z)):
             st.status |= ST_NONFINITE
             continue
-        st.expanded.add(n)
         V = len(z)
         sc.append(row_scores(st.logp[n], z, tau))
         pa.append(np.full(V, n, dtype=np.int64))

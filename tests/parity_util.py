@@ -1,0 +1,84 @@
+"""Comparison helpers shared by the GPU parity tests.
+
+Tolerances:
+* integer outputs (paths, tokens, node sets) are compared exactly, except
+  where the oracle reports a decision within NEAR of its threshold (accept
+  tests |u - ratio|, inverse-CDF margins relative to the row sum, expansion
+  score gaps in nats): those cases are counted and only checked for
+  validity;
+* bf16 attention: max-abs <= 2e-2 and relative L2 <= 5e-3 against the fp64
+  oracle; fp32 attention: max-abs <= 2e-5 and relative L2 <= 2e-6 (fp32
+  accumulation over at most a few hundred terms of unit scale).
+"""
+
+import numpy as np
+import torch
+
+NEAR = 1e-6
+BF16_MAX_ABS, BF16_REL_L2 = 2e-2, 5e-3
+FP32_MAX_ABS, FP32_REL_L2 = 2e-5, 2e-6
+
+
+def cuda(x):
+    return None if x is None else x.to("cuda")
+
+
+def attn_errors(gpu_out, ref_out, mask):
+    """max-abs and relative-L2 error over the rows selected by mask [B][T]."""
+    g = gpu_out.double().cpu().numpy()[mask]
+    r = ref_out[mask]
+    diff = g - r
+    max_abs = float(np.max(np.abs(diff))) if diff.size else 0.0
+    rel = float(np.linalg.norm(diff) / max(np.linalg.norm(r), 1e-300)) if diff.size else 0.0
+    return max_abs, rel
+
+
+def check_attn(gpu_out, ref, dtype, lse_gpu=None, rows_mask=None, poison=None):
+    """Compare a GPU attention result with the oracle dict `ref`."""
+    written = ref["written"] if rows_mask is None else (ref["written"] & rows_mask)
+    valid = ref["valid"] & written
+    max_abs, rel = attn_errors(gpu_out, ref["out"], valid)
+    if dtype == torch.bfloat16:
+        assert max_abs <= BF16_MAX_ABS and rel <= BF16_REL_L2, (max_abs, rel)
+    else:
+        assert max_abs <= FP32_MAX_ABS and rel <= FP32_REL_L2, (max_abs, rel)
+    g = gpu_out.double().cpu().numpy()
+    inval = written & ~ref["valid"]
+    if inval.any():
+        assert np.all(np.isnan(g[inval]))
+    if poison is not None and rows_mask is None:
+        unw = ~ref["written"]
+        if unw.any():
+            assert np.all(g[unw] == poison)
+    if lse_gpu is not None:
+        lg = lse_gpu.double().cpu().numpy()
+        d = np.abs(lg[valid] - ref["lse"][valid])
+        assert (d.max() if d.size else 0.0) <= (2e-3 if dtype == torch.bfloat16 else 2e-5), d.max()
+    return max_abs, rel
+
+
+def check_accept(gpu, ref, parent, T):
+    """Exact comparison of acceptance outputs per sequence; sequences whose
+    oracle walk met a decision within NEAR of its threshold are only
+    checked for validity.  Returns (exact, near)."""
+    n_acc = gpu["n_accepted"].cpu().numpy()
+    acc = gpu["accepted_nodes"].cpu().numpy()
+    tok = gpu["out_tokens"].cpu().numpy()
+    par = parent.cpu().numpy() if isinstance(parent, torch.Tensor) else np.asarray(parent)
+    exact = near = 0
+    for b in range(len(n_acc)):
+        if ref["min_margin"][b] < NEAR:
+            near += 1
+            k = int(n_acc[b])
+            assert 0 <= k <= T
+            c = 0
+            for j in acc[b, :k]:
+                assert par[b, j] == c
+                c = int(j)
+            assert np.all(acc[b, k:] == -1)
+            continue
+        exact += 1
+        assert int(n_acc[b]) == int(ref["n_accepted"][b]), (b, n_acc[b], ref["n_accepted"][b])
+        np.testing.assert_array_equal(acc[b], ref["accepted_nodes"][b])
+        np.testing.assert_array_equal(tok[b], ref["out_tokens"][b])
+    return exact, near

@@ -1,0 +1,190 @@
+"""GPU parity of tree_verify_attn against the fp64 oracle (through the C ABI).
+
+bf16: max-abs <= 2e-2 and relative L2 <= 5e-3; fp32: max-abs <= 2e-5 and
+relative L2 <= 2e-6.  Small cases compare every row (several tiles, ragged
+tails, malformed trees, rows past n_nodes left untouched); the full-size
+workloads compare sampled nodes, computed one by one by the oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle.attention import tree_verify_attn as oracle_attn, ST_BAD_PARENT, ST_BAD_LEN
+from synth import (attn_case, config_attn_case, tree_binary, tree_chain, tree_star,
+                   tree_bfs_fanout, tree_random_recursive, tree_random_depth_limited, CONFIGS)
+from parity_util import check_attn, cuda
+
+pytestmark = pytest.mark.gpu
+POISON = 777.0
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from tree_verification_verify_b200 import build
+    build.build()
+
+
+def _gpu(case, n_nodes=None, prefix_len=None, sparse_topk=None, want_sel=False, q=None):
+    import tree_verification_verify_b200 as tv
+    qd = cuda(case.q if q is None else q)
+    B, T, Hq, d = qd.shape
+    out = torch.full((B, T, Hq, d), POISON, dtype=qd.dtype, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nn = n_nodes if n_nodes is not None else case.n_nodes
+    pl = prefix_len if prefix_len is not None else case.prefix_len
+    k = case.sparse_topk if sparse_topk is None else sparse_topk
+    o, lse, sel = tv.tree_verify_attn(qd, cuda(case.k_cache), cuda(case.v_cache), cuda(pl),
+                                      cuda(case.k_tree), cuda(case.v_tree), cuda(case.parent),
+                                      n_nodes=cuda(nn), scale=case.scale, sparse_topk=k,
+                                      block_size=case.block_size, out=out, want_sel=want_sel,
+                                      dev_status=st)
+    torch.cuda.synchronize()
+    return o, lse, sel, int(st.item())
+
+
+def _oracle(case, n_nodes=None, prefix_len=None, rows=None, sparse_topk=None):
+    return oracle_attn(case.q, case.k_cache, case.v_cache,
+                       case.prefix_len if prefix_len is None else prefix_len,
+                       case.k_tree, case.v_tree, case.parent,
+                       n_nodes=case.n_nodes if n_nodes is None else n_nodes, scale=case.scale,
+                       sparse_topk=case.sparse_topk if sparse_topk is None else sparse_topk,
+                       block_size=case.block_size, rows=rows)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_tiny_config_fp32(seed):
+    case = config_attn_case("tiny", seed=seed)
+    o, lse, _, st = _gpu(case)
+    ref = _oracle(case)
+    check_attn(o, ref, torch.float32, lse_gpu=lse, poison=POISON)
+    assert st == 0
+
+
+SHAPES = [
+    # B, T, Hq, Hkv, d, L, dtype, tree
+    (2, 23, 8, 2, 64, [300, 0], "bf16", "recursive"),
+    (1, 40, 32, 8, 128, [1000], "bf16", "bfs"),
+    (3, 17, 4, 4, 128, [129, 64, 1], "bf16", "depth6"),
+    (1, 9, 16, 1, 64, [513], "bf16", "chain"),
+    (2, 33, 8, 1, 32, [77, 200], "fp32", "star"),
+    (1, 15, 64, 8, 128, [2048], "bf16", "binary"),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[f"{s[6]}-T{s[1]}-G{s[2]//s[3]}-d{s[4]}" for s in SHAPES])
+def test_shapes(shape):
+    B, T, Hq, Hkv, d, L, dtype, tree = shape
+    g = torch.Generator().manual_seed(T)
+    par = {"recursive": tree_random_recursive(T, g), "bfs": tree_bfs_fanout(T, (4, 3, 2)),
+           "depth6": tree_random_depth_limited(T, 6, g), "chain": tree_chain(T),
+           "star": tree_star(T), "binary": tree_binary(T)}[tree]
+    case = attn_case(B, T, Hq, Hkv, d, L, dtype, par, seed=B * T)
+    o, lse, _, st = _gpu(case)
+    ref = _oracle(case)
+    check_attn(o, ref, o.dtype, lse_gpu=lse, poison=POISON)
+    assert st == ref["status"] == 0
+
+
+def test_partial_trees_and_malformed_input():
+    T = 21
+    par = tree_random_recursive(T, torch.Generator().manual_seed(2))
+    par[13] = 17                                      # malformed: 17 >= 13
+    case = attn_case(3, T, 8, 2, 128, [250, 40, 3], "bf16", par, seed=5, n_nodes=[21, 9, 0])
+    o, lse, _, st = _gpu(case)
+    ref = _oracle(case)
+    check_attn(o, ref, torch.bfloat16, lse_gpu=lse, poison=POISON)
+    assert st == ref["status"] and st & ST_BAD_PARENT
+    bad_pl = torch.tensor([250, 999, 3], dtype=torch.int32)
+    bad_nn = torch.tensor([21, 9, 30], dtype=torch.int32)
+    o, lse, _, st = _gpu(case, n_nodes=bad_nn, prefix_len=bad_pl)
+    ref = _oracle(case, n_nodes=bad_nn, prefix_len=bad_pl)
+    check_attn(o, ref, torch.bfloat16, poison=POISON)
+    assert st == ref["status"] and st & ST_BAD_LEN
+
+
+def test_strided_query_view():
+    T, Hq, d = 12, 8, 64
+    case = attn_case(2, T, Hq, 2, d, [100, 31], "bf16", tree_binary(T), seed=3)
+    big = torch.randn(2, T, Hq + 3, d + 64).to(torch.bfloat16)
+    big[:, :, 1:Hq + 1, 32:32 + d] = case.q
+    qv = big[:, :, 1:Hq + 1, 32:32 + d]                 # non-contiguous heads / rows
+    o, lse, _, st = _gpu(case, q=qv)
+    ref = _oracle(case)
+    check_attn(o, ref, torch.bfloat16, lse_gpu=lse)
+
+
+def _sample_rows(B, T, per_b, seed):
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for b in range(B):
+        for i in rng.choice(T, size=min(per_b, T), replace=False):
+            rows.add((b, int(i)))
+        rows.add((b, 0))
+        rows.add((b, T - 1))
+    return rows
+
+
+def _rows_mask(rows, B, T):
+    m = np.zeros((B, T), dtype=bool)
+    for b, i in rows:
+        m[b, i] = True
+    return m
+
+
+@pytest.mark.parametrize("name,per_b", [("llama3_8b", 64), ("specexec70b", 24), ("serving", 2), ("longctx", 3)])
+def test_full_size_dense_sampled(name, per_b):
+    c = CONFIGS[name]
+    case = config_attn_case(name, seed=0)
+    o, lse, _, st = _gpu(case)
+    rows = _sample_rows(c["B"], c["T"], per_b, 1)
+    ref = _oracle(case, rows=rows)
+    check_attn(o, ref, torch.bfloat16, lse_gpu=lse, rows_mask=_rows_mask(rows, c["B"], c["T"]))
+    assert st == 0
+
+
+def test_sparse_small_all_blocks_equals_dense():
+    T = 13
+    case = attn_case(2, T, 8, 2, 128, [300, 64], "bf16", tree_binary(T), seed=4)
+    od, _, _, _ = _gpu(case, sparse_topk=0)
+    os_, _, sel, st = _gpu(case, sparse_topk=5, want_sel=True)
+    ref = _oracle(case, sparse_topk=5)
+    check_attn(os_, ref, torch.bfloat16, poison=POISON)
+    assert torch.equal(sel.cpu(), torch.from_numpy(ref["sel"]).to(torch.int32))
+    assert (od.float() - os_.float()).abs().max().item() < 2e-2
+
+
+def _check_sparse(case, rows, B, T, Hkv, G, k):
+    o, lse, sel, st = _gpu(case, want_sel=True)
+    ref = _oracle(case, rows=rows)
+    sel = sel.cpu().numpy()
+    checked = near = 0
+    for (b, i) in rows:
+        for g in range(Hkv):
+            if not np.array_equal(sel[b, i, g], ref["sel"][b, i, g]):
+                # only an fp32 near-tie at the k-th block may differ
+                assert ref["sel_gap"][b, i, g] < 1e-4, (b, i, g, ref["sel_gap"][b, i, g])
+                near += 1
+                continue
+            hs = slice(g * G, (g + 1) * G)
+            got = o[b, i, hs].double().cpu().numpy()
+            want = ref["out"][b, i, hs]
+            assert np.max(np.abs(got - want)) <= 2e-2
+            checked += 1
+    assert checked > 0
+    return checked, near, st
+
+
+def test_sparse_small_offsets():
+    T, L, bs = 20, 64 * 60, 64
+    case = attn_case(2, T, 8, 2, 128, [L, L - 37], "bf16", tree_bfs_fanout(T, (4, 3, 2)), seed=6,
+                     offset_frac=0.1, block_size=bs, sparse_topk=8)
+    rows = {(b, i) for b in range(2) for i in range(T)}
+    _check_sparse(case, rows, 2, T, 2, 4, 8)
+
+
+def test_full_size_sparse_sampled():
+    c = CONFIGS["longctx"]
+    case = config_attn_case("longctx", seed=0, sparse=True)
+    rows = _sample_rows(c["B"], c["T"], 3, 2)
+    checked, near, st = _check_sparse(case, rows, c["B"], c["T"], c["Hkv"], c["Hq"] // c["Hkv"], 32)
+    assert st == 0

@@ -1,0 +1,144 @@
+"""GPU parity of tree_expand_topb against the fp64 oracle (through the C ABI).
+
+Each round's appended nodes (parent, token, order) must be identical and the
+cumulative log-probabilities agree to 1e-9; once the oracle reports a score
+gap below 1e-6 nats among the ranks that decided a round, the remaining
+rounds are not compared (counted as near-ties)."""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle.expand import ExpandState as OState, expand_call
+from synth import expand_case, CONFIGS
+from parity_util import NEAR
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "expand_worked_example.txt")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from tree_verification_verify_b200 import build
+    build.build()
+
+
+def _compare_build(V, Bsel, budget, logits_fn, tau=1.0, root_token=0):
+    """Run GPU and oracle round by round on identical rows.  logits_fn(call,
+    R) returns [R][V] fp32 rows for the frontier of that call (identical
+    frontiers on both sides, checked every round)."""
+    import tree_verification_verify_b200 as tv
+    st = tv.tree_expand_init(budget, V, Bsel, root_token=root_token)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    os_ = OState(budget, root_token)
+    frontier = [0]
+    call = 0
+    compared = 0
+    near = False
+    while os_.n_nodes < budget and frontier:
+        z = logits_fn(call, len(frontier))
+        rows = torch.tensor(frontier, dtype=torch.int32, device="cuda")
+        tv.tree_expand_topb(st, z.cuda(), rows, draft_temperature=tau, dev_status=status)
+        new = expand_call(os_, z, frontier, Bsel, tau)
+        torch.cuda.synchronize()
+        gap = os_.gaps[-1]
+        nap = int(st.n_appended.item())
+        gf = st.frontier.cpu().numpy()[:nap].tolist()
+        if gap < NEAR:
+            near = True
+            break
+        assert nap == len(new), (call, nap, len(new))
+        assert gf == new
+        n = os_.n_nodes
+        gp = st.parent.cpu().numpy()[:n]
+        gt = st.token.cpu().numpy()[:n]
+        gl = st.logp.cpu().numpy()[:n]
+        np.testing.assert_array_equal(gp, np.array(os_.parent))
+        np.testing.assert_array_equal(gt, np.array(os_.token))
+        np.testing.assert_allclose(gl, np.array(os_.logp), rtol=0, atol=1e-9)
+        frontier = new
+        call += 1
+        compared += 1
+    assert int(status.item()) == os_.status
+    return compared, near, st, os_
+
+
+def test_tiny_config():
+    ec = expand_case(256, 8, 64, 3.0, seed=0)
+    compared, near, st, os_ = _compare_build(ec.V, ec.Bsel, ec.budget, lambda c, R: ec.round_logits(c, R))
+    assert not near and os_.n_nodes == 64 and compared == ec.n_calls()
+
+
+@pytest.mark.parametrize("V,Bsel,budget,sigma,tau", [
+    (3, 4, 20, 1.0, 1.0),        # few candidates per row: the pool carries the rounds
+    (1, 2, 9, 1.0, 1.0),         # one token: a chain
+    (37, 5, 101, 2.0, 0.7),      # ragged vocabulary, temperature
+    (5000, 200, 1200, 4.0, 1.0), # Bsel above one merge sub-step
+    (700, 128, 2048, 4.0, 1.3),  # lists shorter than the remaining budget
+])
+def test_shapes(V, Bsel, budget, sigma, tau):
+    ec = expand_case(V, Bsel, budget, sigma, seed=V)
+    compared, near, st, os_ = _compare_build(V, Bsel, budget, lambda c, R: ec.round_logits(c, R), tau=tau)
+    assert compared >= 1
+
+
+def test_worked_example():
+    ln3 = math.log(3.0)
+    rows = {(): [0.0, ln3], (1,): [ln3, 0.0], (0,): [0.0, ln3], (1, 0): [0.0, 0.0]}
+    import tree_verification_verify_b200 as tv
+    for case, Bsel, budget in (("A", 1, 4), ("B", 2, 5)):
+        st = tv.tree_expand_init(budget, 2, Bsel)
+        paths = {0: ()}
+        frontier = [0]
+        while frontier:
+            z = torch.tensor([rows[paths[n]] for n in frontier], dtype=torch.float32)
+            tv.tree_expand_topb(st, z.cuda(), torch.tensor(frontier, dtype=torch.int32, device="cuda"))
+            k = int(st.n_appended.item())
+            frontier = st.frontier.cpu().tolist()[:k]
+            par = st.parent.cpu().tolist()
+            tok = st.token.cpu().tolist()
+            for n in frontier:
+                paths[n] = paths[par[n]] + (tok[n],)
+            frontier = [n for n in frontier if paths[n] in rows]
+            if int(st.n_nodes.item()) >= budget:
+                break
+        want = []
+        for line in open(GOLDEN):
+            if line.startswith(case + " "):
+                _, node, parent, token, prob = line.split()
+                want.append((int(node), int(parent), int(token), prob))
+        par = st.parent.cpu().tolist()
+        tok = st.token.cpu().tolist()
+        lp = st.logp.cpu().tolist()
+        from fractions import Fraction
+        for node, parent, token, prob in want:
+            assert par[node] == parent and tok[node] == token
+            assert abs(lp[node] - math.log(float(Fraction(prob)))) < 1e-7
+
+
+def test_bad_rows_and_nonfinite():
+    import tree_verification_verify_b200 as tv
+    st = tv.tree_expand_init(16, 8, 4)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    z = torch.randn(3, 8, device="cuda")
+    tv.tree_expand_topb(st, z, torch.tensor([0, 5, -1], dtype=torch.int32, device="cuda"), dev_status=status)
+    assert int(st.n_appended.item()) == 4 and status.item() & 8
+    status.zero_()
+    z2 = torch.randn(2, 8, device="cuda")
+    z2[1, 3] = float("inf")
+    f = st.frontier[:2].clone()
+    tv.tree_expand_topb(st, z2, f, dev_status=status)
+    assert status.item() & 4
+    assert int(st.n_nodes.item()) == 9
+
+
+def test_specexec70b_full_build():
+    c = CONFIGS["specexec70b"]
+    ec = expand_case(c["V"], c["Bsel"], c["budget"], c["sigma"], seed=0)
+    compared, near, st, os_ = _compare_build(ec.V, ec.Bsel, ec.budget, lambda k, R: ec.round_logits(k, R))
+    assert compared >= 8
+    if not near:
+        assert compared == ec.n_calls() == 16

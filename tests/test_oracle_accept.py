@@ -180,6 +180,7 @@ def _check_lossless(par, V, tau, mode, seed=0, sigma=1.0):
     the path-keyed target."""
     T = len(par)
     kids_order = list(range(1, T))
+    tau = float(np.float32(tau))        # the walk takes an fp32 temperature
 
     def target_p(path):
         return softmax_t(_path_row(path, 1, V, sigma, seed), tau)
