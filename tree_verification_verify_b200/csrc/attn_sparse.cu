@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(AttnParams p)
       int taken = 0, w = 0, ties = 0;
       for (int j = 0; j < nblk; ++j) {
         const uint32_t key = ~f32_key(sc[j]);
-        if (key < theta || (key == theta && ties < need)) {
+        if ((key < theta || (key == theta && ties < need)) && w < k) {
           if (key == theta) ++ties;
           sel[w++] = j;
           ++taken;

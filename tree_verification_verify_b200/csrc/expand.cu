@@ -99,6 +99,7 @@ struct RowShared {
 __device__ void find_rank_bin(const uint32_t* hist, int nbins, int rank, int* bin,
                               int* before, RowShared& sh) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) { sh.bc[0] = 0; sh.bc[1] = 0; }
   const int per = (nbins + blockDim.x - 1) / blockDim.x;
   const int lo = min(tid * per, nbins), hi = min(lo + per, nbins);
   int ls = 0;
@@ -269,7 +270,7 @@ expand_rows_kernel(ExpandParams p) {
     const uint32_t k = zdesc_key(__ldg(row + e));
     if (k < theta || (k == theta && n_eq == need)) {
       const int pos = atomicAdd(&s_count, 1);
-      sbuf[pos] = (static_cast<uint64_t>(k) << 32) | static_cast<uint32_t>(e);
+      if (pos < K) sbuf[pos] = (static_cast<uint64_t>(k) << 32) | static_cast<uint32_t>(e);
     }
   }
   __syncthreads();
@@ -297,7 +298,7 @@ expand_rows_kernel(ExpandParams p) {
       const int rank = taken + sh.red_i[warp] + __popc(m & ((1u << lane) - 1u));
       if (is && rank < need) {
         const int pos = atomicAdd(&s_count, 1);
-        sbuf[pos] = (static_cast<uint64_t>(theta) << 32) | static_cast<uint32_t>(e);
+        if (pos < K) sbuf[pos] = (static_cast<uint64_t>(theta) << 32) | static_cast<uint32_t>(e);
       }
       taken += sh.bc[3];
       __syncthreads();
@@ -444,9 +445,12 @@ expand_merge_kernel(ExpandParams p) {
     if (H > s) radix_select_ab(A, Bk, H, s, &tA, &tB, sh);
     __syncthreads();
     for (int i = tid; i < H; i += blockDim.x)
-      if (comp_le(A[i], Bk[i], tA, tB)) sh.qlist[atomicAdd(&sh.cnt[1], 1)] = static_cast<int>(Bk[i] >> 18);
+      if (comp_le(A[i], Bk[i], tA, tB)) {
+        const int k = atomicAdd(&sh.cnt[1], 1);
+        if (k < kMergeStep) sh.qlist[k] = static_cast<int>(Bk[i] >> 18);
+      }
     __syncthreads();
-    const int Q = sh.cnt[1];
+    const int Q = min(sh.cnt[1], kMergeStep);
     // 2. candidates ranked within the first s heads' bound, <= s per list
     for (int qi = warp; qi < Q; qi += kMergeWarps) {
       const int nd = sh.qlist[qi];
@@ -473,14 +477,16 @@ expand_merge_kernel(ExpandParams p) {
         off = __shfl_sync(0xffffffffu, off, 0);
         if (ok) {
           const int k = __popc(m & ((1u << lane) - 1u));
-          A[off + k] = a;   // heads are no longer needed
-          Bk[off + k] = bb;
+          if (off + k < kMergeCap) {
+            A[off + k] = a;   // heads are no longer needed
+            Bk[off + k] = bb;
+          }
         }
         if (c < 32) break;
       }
     }
     __syncthreads();
-    const int C = sh.cnt[2];
+    const int C = min(sh.cnt[2], kMergeCap);
     uint64_t uA = ~0ull;
     uint32_t uB = ~0u;
     if (C > s) radix_select_ab(A, Bk, C, s, &uA, &uB, sh);
@@ -489,11 +495,13 @@ expand_merge_kernel(ExpandParams p) {
     for (int i = tid; i < C; i += blockDim.x)
       if (comp_le(A[i], Bk[i], uA, uB)) {
         const int k = atomicAdd(&sh.cnt[3], 1);
-        sh.selA[k] = A[i];
-        sh.selB[k] = Bk[i];
+        if (k < kMergeStep) {
+          sh.selA[k] = A[i];
+          sh.selB[k] = Bk[i];
+        }
       }
     __syncthreads();
-    const int S = sh.cnt[3];
+    const int S = min(sh.cnt[3], kMergeStep);
     for (int i = S + tid; i < kMergeStep; i += blockDim.x) { sh.selA[i] = ~0ull; sh.selB[i] = ~0u; }
     __syncthreads();
     // 3. sort the winners by (score desc, parent asc, token asc)
