@@ -1,8 +1,9 @@
 """GPU parity of tree_expand_topb against the fp64 oracle (through the C ABI).
 
 Each round's appended nodes (parent, token, order) must be identical and the
-cumulative log-probabilities agree to 1e-9; once the oracle reports a score
-gap below 1e-6 nats among the ranks that decided a round, the remaining
+cumulative log-probabilities agree to 1e-12 (fp64 scores from fp64
+exponentials on both sides); once the oracle reports a score
+gap below 1e-10 nats among the ranks that decided a round, the remaining
 rounds are not compared (counted as near-ties)."""
 
 import math
@@ -14,7 +15,11 @@ import torch
 
 from oracle.expand import ExpandState as OState, expand_call
 from synth import expand_case, CONFIGS
-from parity_util import NEAR
+
+# Both sides score candidates in fp64 from fp64 exponentials, so their
+# scores differ by a few ulps per tree level; ranks closer than this many
+# nats are counted as near-ties.
+NEAR = 1e-10
 
 pytestmark = pytest.mark.gpu
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "expand_worked_example.txt")
@@ -58,7 +63,7 @@ def _compare_build(V, Bsel, budget, logits_fn, tau=1.0, root_token=0):
         gl = st.logp.cpu().numpy()[:n]
         np.testing.assert_array_equal(gp, np.array(os_.parent))
         np.testing.assert_array_equal(gt, np.array(os_.token))
-        np.testing.assert_allclose(gl, np.array(os_.logp), rtol=0, atol=1e-9)
+        np.testing.assert_allclose(gl, np.array(os_.logp), rtol=0, atol=1e-12)
         frontier = new
         call += 1
         compared += 1

@@ -196,10 +196,12 @@ expand_rows_kernel(ExpandParams p) {
       }
     const float wm = warp_max(m4);
     double a = 0.0;
+    // double-precision exponentials: the row's lse enters every cumulative
+    // score, and cross-row ranks must not move by more than fp64 rounding
 #pragma unroll
     for (int k = 0; k < 4; ++k)
       if (e0 + k < V && isfinite(xs[k]))
-        a += exp_neg((static_cast<double>(xs[k]) - static_cast<double>(wm)) * invtau);
+        a += exp((static_cast<double>(xs[k]) - static_cast<double>(wm)) * invtau);
     a = warp_sum(a);
     if (lane == 0) { seg_m[s] = wm; seg_s[s] = a; }
     lmax = fmaxf(lmax, wm);
