@@ -83,7 +83,9 @@ enum {
   TV_DEV_BAD_TOKEN = 2,     /* a draft token outside [0, V)                */
   TV_DEV_NONFINITE = 4,     /* NaN/Inf logits, or invalid probabilities    */
   TV_DEV_BAD_ROW = 8,       /* expansion row for a missing/expanded node   */
-  TV_DEV_BAD_LEN = 16       /* n_nodes or prefix_len out of range          */
+  TV_DEV_BAD_LEN = 16,      /* n_nodes or prefix_len out of range          */
+  TV_DEV_TIMEOUT = 32       /* a bounded in-kernel wait expired; the       */
+                            /* affected outputs are NaN                    */
 };
 
 typedef enum { TV_FP32 = 0, TV_BF16 = 1 } tv_dtype;
@@ -271,6 +273,10 @@ TV_API tv_status tree_expand_topb(const tv_expand_args* a, void* ws, size_t ws_b
 /* ------------------------------------------------------------------------
  * Utilities
  * ---------------------------------------------------------------------- */
+/* Which kernels tree_verify_attn would run for these arguments:
+ * 0 = CUDA-core split-KV, 1 = tcgen05 tensor-core prefix kernel,
+ * 2 = block top-k sparse path, -1 = the arguments are rejected. */
+TV_API int32_t tv_attn_path(const tv_attn_args* a);
 /* Library version, e.g. "treeverify 0.1.0 sm_100a". */
 TV_API const char* tree_verify_version(void);
 /* Static text for a tv_status value. */

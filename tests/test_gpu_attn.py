@@ -68,6 +68,7 @@ SHAPES = [
     (1, 9, 16, 1, 64, [513], "bf16", "chain"),
     (2, 33, 8, 1, 32, [77, 200], "fp32", "star"),
     (1, 15, 64, 8, 128, [2048], "bf16", "binary"),
+    (2, 70, 16, 2, 128, [0, 700], "bf16", "recursive"),
 ]
 
 
@@ -80,6 +81,9 @@ def test_shapes(shape):
            "star": tree_star(T), "binary": tree_binary(T)}[tree]
     case = attn_case(B, T, Hq, Hkv, d, L, dtype, par, seed=B * T)
     o, lse, _, st = _gpu(case)
+    import tree_verification_verify_b200 as tv
+    # bf16 with d = 128 and a power-of-two group runs the tensor-core kernel
+    assert tv.last_attn_path == (1 if (dtype == "bf16" and d == 128) else 0)
     ref = _oracle(case)
     check_attn(o, ref, o.dtype, lse_gpu=lse, poison=POISON)
     assert st == ref["status"] == 0
@@ -136,6 +140,8 @@ def test_full_size_dense_sampled(name, per_b):
     c = CONFIGS[name]
     case = config_attn_case(name, seed=0)
     o, lse, _, st = _gpu(case)
+    import tree_verification_verify_b200 as tv
+    assert tv.last_attn_path == 1
     rows = _sample_rows(c["B"], c["T"], per_b, 1)
     ref = _oracle(case, rows=rows)
     check_attn(o, ref, torch.bfloat16, lse_gpu=lse, rows_mask=_rows_mask(rows, c["B"], c["T"]))

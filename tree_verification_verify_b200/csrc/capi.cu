@@ -111,6 +111,12 @@ extern "C" size_t tree_verify_attn_workspace_size(const tv_attn_args* a) {
   return plan_attn(a).total;
 }
 
+extern "C" int32_t tv_attn_path(const tv_attn_args* a) {
+  if (check_attn(a) != TV_OK) return -1;
+  const AttnPlan pl = plan_attn(a);
+  return pl.sparse ? 2 : (pl.tc ? 1 : 0);
+}
+
 extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws_bytes,
                                       tv_stream_t stream) {
   const tv_status st = check_attn(a);
