@@ -1,4 +1,4 @@
-// tree_accept kernels: per-node decisions over vocabulary rows, then a walk
+// tree_accept kernel: per-node decisions over vocabulary rows, then a walk
 // from the root along the accepted children.
 //
 // Acceptance rules (SpecExec page, "Approach" and "Builds on": speculative
@@ -10,18 +10,27 @@
 //   SPECEXEC    x ~ softmax(z_c / tau) by inverse CDF, descend to a child
 //               carrying x.
 // Every node's decision depends only on its own rows and its own Philox
-// draws, so all nodes decide in parallel (one CTA per node row) and a
-// second, tiny kernel follows the decisions from the root.
+// draws, so all nodes decide in parallel; the last node of a sequence to
+// finish (an atomic ticket, no waiting) walks the decisions from the root.
 //
-// Data layout of a row pass: the row is cut into 128-element segments; a
-// warp owns a segment (lane l holds elements 4l..4l+3, one 16-byte load).
+// Layout of a row pass.  A thread-block cluster of C CTAs (C <= 8) owns one
+// node row; CTA rank r owns a contiguous slice of 128-element segments.  A
+// warp owns a segment (lane l holds elements 4l..4l+3, one 16-byte load) and
+// keeps four segments in flight.  Cross-CTA sums and maxima go through
+// distributed shared memory (double-buffered slots, one cluster barrier per
+// reduction); every CTA of the cluster computes the same reduced values and
+// so takes the same branches.
+//
 // Per segment the first pass keeps the segment maximum wm and the sum of
-// exp((z - wm)/tau); element weights are always recomputed in that same
-// segment frame, scaled by f_seg = exp((wm - M)/tau) (M the row maximum),
-// so segment sums and element values agree to rounding order.  Residuals
+// exp((z - wm)/tau); element weights are recomputed in that same segment
+// frame, scaled by f_seg = exp((wm - M)/tau) (M the row maximum).  Residuals
 // are parametrised as r = (p - c q)^+ / D: rejecting a child with the
 // current (c, D) gives c' = c + D and D' = sum_t (p - c' q)^+, one pass.
+#include <cooperative_groups.h>
+
 #include "tv_common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace tv {
 
@@ -45,26 +54,44 @@ struct AcceptParams {
   uint64_t seed, step;
   uint32_t* status;
   AcceptDec* dec;           // [B][T]
+  int32_t* ticket;          // [B], zero between calls
   int32_t* n_acc;
   int32_t* acc_nodes;
   int32_t* out_tokens;
   double* min_margin;
+  int C;                    // CTAs per row (cluster size)
+  int seg_per_cta;          // 128-element segments per CTA
 };
 
 constexpr int kAcceptThreads = 512;
 constexpr int kAcceptWarps = kAcceptThreads / kWarp;
 constexpr int kSeg = 128;
+constexpr int kUnroll = 2;
+constexpr int kMaxSegPerCta = 512;      // 65536 elements per CTA
 
-// ------------------------------------------------------------ block helpers
+// ------------------------------------------------------------ shared state
+
+struct Slot {            // one CTA's contribution to a cluster reduction
+  double a, b;
+  float f;
+  int i, j;
+};
 
 struct AcceptShared {
   double red_d[kAcceptWarps];
   float red_f[kAcceptWarps];
   int red_i[kAcceptWarps];
+  int red_j[kAcceptWarps];
   int wofs[kAcceptWarps];
   int clist[kAcceptThreads];
   int bc_int[4];
   double bc_dbl[4];
+  Slot slot[2];
+  double rank_tot[8];      // per-CTA totals of the current weights
+  float seg_m[kMaxSegPerCta];
+  double seg_f[kMaxSegPerCta];
+  double seg_w[kMaxSegPerCta];
+  double seg_r[kMaxSegPerCta];
 };
 
 __device__ __forceinline__ double block_sum_d(double v, AcceptShared& sh) {
@@ -73,29 +100,13 @@ __device__ __forceinline__ double block_sum_d(double v, AcceptShared& sh) {
   __syncthreads();
   if (lane == 0) sh.red_d[warp] = v;
   __syncthreads();
-  double t = 0.0;
   if (warp == 0) {
-    t = (lane < kAcceptWarps) ? sh.red_d[lane] : 0.0;
+    double t = (lane < kAcceptWarps) ? sh.red_d[lane] : 0.0;
     t = warp_sum(t);
     if (lane == 0) sh.bc_dbl[0] = t;
   }
   __syncthreads();
   return sh.bc_dbl[0];
-}
-
-__device__ __forceinline__ float block_max_f(float v, AcceptShared& sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = warp_max(v);
-  __syncthreads();
-  if (lane == 0) sh.red_f[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    float t = (lane < kAcceptWarps) ? sh.red_f[lane] : -INFINITY;
-    t = warp_max(t);
-    if (lane == 0) sh.red_f[0] = t;
-  }
-  __syncthreads();
-  return sh.red_f[0];
 }
 
 __device__ __forceinline__ int block_min_i(int v, AcceptShared& sh) {
@@ -115,9 +126,34 @@ __device__ __forceinline__ int block_min_i(int v, AcceptShared& sh) {
   return sh.bc_int[0];
 }
 
+// Cluster all-gather of one Slot per CTA: after the call every thread of
+// every CTA sees the C slots in `out` (rank order).  `k` counts the
+// reductions so that consecutive ones use alternate slots.
+__device__ __forceinline__ void cluster_gather(cg::cluster_group& cl, AcceptShared& sh, const Slot& mine,
+                                               int C, int& k, Slot* out) {
+  Slot* s = &sh.slot[k & 1];
+  if (threadIdx.x == 0) *s = mine;
+  cl.sync();
+  for (int r = 0; r < C; ++r) {
+    const Slot* rs = cl.map_shared_rank(s, r);
+    out[r] = *rs;
+  }
+  ++k;
+}
+
+// Weight of one element in the current distribution: e = exp((z-wm)/tau) *
+// f_seg (unnormalised softmax), or the residual (e/s - c q)^+.
+__device__ __forceinline__ double elem_weight(float z, float q, float wm, double fseg, double invtau,
+                                              double inv_s, double cpar, bool resid) {
+  const double e = exp_neg((static_cast<double>(z) - static_cast<double>(wm)) * invtau) * fseg;
+  if (!resid) return e;
+  const double w = e * inv_s - cpar * static_cast<double>(q);
+  return w > 0.0 ? w : 0.0;
+}
+
 // Lowest-index child of c (c < j < n) that carries token x, or -1.
-__device__ int first_child_with_token(const int32_t* par, const int32_t* tok, int c, int n,
-                                      int x, AcceptShared& sh) {
+__device__ int first_child_with_token(const int32_t* par, const int32_t* tok, int c, int n, int x,
+                                      AcceptShared& sh) {
   int best = INT_MAX;
   for (int j = c + 1 + threadIdx.x; j < n; j += blockDim.x)
     if (par[j] == c && tok[j] == x) { best = j; break; }
@@ -125,163 +161,205 @@ __device__ int first_child_with_token(const int32_t* par, const int32_t* tok, in
   return best == INT_MAX ? -1 : best;
 }
 
-// Weight of one element in the current distribution: e = exp((z-wm)/tau) *
-// f_seg (unnormalised softmax), or the residual (e/s - c q)^+.
-__device__ __forceinline__ double elem_weight(float z, float q, float wm, double fseg,
-                                              double invtau, double inv_s, double cpar,
-                                              bool resid) {
-  const double e = exp_neg((static_cast<double>(z) - static_cast<double>(wm)) * invtau) * fseg;
-  if (!resid) return e;
-  const double w = e * inv_s - cpar * static_cast<double>(q);
-  return w > 0.0 ? w : 0.0;
-}
-
-// Inverse-CDF sample: smallest t with sum_{s<=t} w_s > u * W over the
-// current weights (segment sums in seg_w).  Returns t and the relative
-// margin min(cum_t - uW, uW - cum_{t-1}) / W.  Called by the whole block.
-__device__ void sample_row(const float* zr, const float* qr, bool zvec, bool qvec, int V,
-                           int nseg, const float* seg_m, const double* seg_f,
-                           const double* seg_w, double invtau, double inv_s, double cpar,
-                           bool resid, double u, int* out_t, double* out_margin,
-                           AcceptShared& sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  double part = 0.0;
-  for (int s = threadIdx.x; s < nseg; s += blockDim.x) part += seg_w[s];
-  const double W = block_sum_d(part, sh);
-  const double target = u * W;
-  if (warp == 0) {
-    // 1. the segment where the running sum first exceeds target
-    const int per = (nseg + 31) / 32;
-    const int lo = min(lane * per, nseg), hi = min(lo + per, nseg);
-    double ls = 0.0;
-    for (int s = lo; s < hi; ++s) ls += seg_w[s];
-    const double incl = warp_incl_scan(ls);
-    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
-    if (lane == 0) excl = 0.0;
-    const unsigned m = __ballot_sync(0xffffffffu, incl > target);
-    int seg = -1;
-    double base = 0.0;
-    if (m != 0u) {
-      const int L = __ffs(m) - 1;
-      if (lane == L) {
-        double cum = excl;
-        int s = lo;
-        for (; s < hi; ++s) {
-          if (cum + seg_w[s] > target) break;
-          cum += seg_w[s];
-        }
-        seg = (s < hi) ? s : hi - 1;
-        base = (s < hi) ? cum : cum - seg_w[hi - 1];
-      }
-      seg = __shfl_sync(0xffffffffu, seg, L);
-      base = __shfl_sync(0xffffffffu, base, L);
-    } else {
-      // target >= total by rounding: the last segment with weight
-      int last = -1;
-      for (int s = lo; s < hi; ++s) if (seg_w[s] > 0.0) last = s;
-      const unsigned mm = __ballot_sync(0xffffffffu, last >= 0);
-      const int L = mm ? 31 - __clz(mm) : 0;
-      seg = __shfl_sync(0xffffffffu, last, L);
-      if (seg < 0) seg = 0;
-      base = -1.0;           // marks "take the last positive element"
-    }
-    // 2. inside the segment
-    const int e0 = seg * kSeg + lane * 4;
-    const float4 zv = load4(zr, e0, V, zvec, -INFINITY);
-    float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (resid) qv = load4(qr, e0, V, qvec, 0.f);
-    const float wm = seg_m[seg];
-    const double fs = seg_f[seg];
-    double w[4];
-    w[0] = (e0 + 0 < V) ? elem_weight(zv.x, qv.x, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
-    w[1] = (e0 + 1 < V) ? elem_weight(zv.y, qv.y, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
-    w[2] = (e0 + 2 < V) ? elem_weight(zv.z, qv.z, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
-    w[3] = (e0 + 3 < V) ? elem_weight(zv.w, qv.w, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
-    int t = -1;
-    double margin = 0.0;
-    if (base >= 0.0) {
-      const double lsum = ((w[0] + w[1]) + w[2]) + w[3];
-      const double li = warp_incl_scan(lsum);
-      double le = __shfl_up_sync(0xffffffffu, li, 1);
-      if (lane == 0) le = 0.0;
-      const unsigned m2 = __ballot_sync(0xffffffffu, base + li > target);
-      if (m2 != 0u) {
-        const int L = __ffs(m2) - 1;
-        if (lane == L) {
-          double cum = base + le;
-          for (int k = 0; k < 4; ++k) {
-            if (cum + w[k] > target) {
-              t = e0 + k;
-              margin = fmin(cum + w[k] - target, target - cum) / W;
-              break;
-            }
-            cum += w[k];
-          }
-        }
-        t = __shfl_sync(0xffffffffu, t, L);
-        margin = __shfl_sync(0xffffffffu, margin, L);
-      }
-    }
-    if (t < 0) {
-      // rounding put the crossing at the segment's end: last positive element
-      int lp = -1;
-      for (int k = 0; k < 4; ++k) if (w[k] > 0.0) lp = e0 + k;
-      const unsigned mm = __ballot_sync(0xffffffffu, lp >= 0);
-      const int L = mm ? 31 - __clz(mm) : 0;
-      t = __shfl_sync(0xffffffffu, lp, L);
-      margin = 0.0;
-    }
-    if (lane == 0) { sh.bc_int[1] = t; sh.bc_dbl[1] = margin; }
-  }
-  __syncthreads();
-  *out_t = sh.bc_int[1];
-  *out_margin = sh.bc_dbl[1];
-  __syncthreads();
-}
-
-// One pass over the row computing the segment sums of the residual
-// weights (e/s - c q)^+; returns their total.
-__device__ double residual_pass(const float* zr, const float* qr, bool zvec, bool qvec, int V,
-                                int nseg, const float* seg_m, const double* seg_f,
-                                double* seg_out, double invtau, double inv_s, double cpar,
-                                AcceptShared& sh) {
+// One pass over this CTA's slice computing the segment sums of the residual
+// weights (e/s - c q)^+ into seg_out; returns the slice total.
+__device__ double residual_pass(const float* zr, const float* qr, bool zvec, bool qvec, int V, int seg0,
+                                int nloc, const AcceptShared& sh, double* seg_out, double invtau, double inv_s,
+                                double cpar, AcceptShared& shw) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   double tot = 0.0;
-  for (int s = warp; s < nseg; s += kAcceptWarps) {
-    const int e0 = s * kSeg + lane * 4;
-    const float4 zv = load4(zr, e0, V, zvec, -INFINITY);
-    const float4 qv = load4(qr, e0, V, qvec, 0.f);
-    const float wm = seg_m[s];
-    const double fs = seg_f[s];
-    double a = 0.0;
-    if (e0 + 0 < V) a += elem_weight(zv.x, qv.x, wm, fs, invtau, inv_s, cpar, true);
-    if (e0 + 1 < V) a += elem_weight(zv.y, qv.y, wm, fs, invtau, inv_s, cpar, true);
-    if (e0 + 2 < V) a += elem_weight(zv.z, qv.z, wm, fs, invtau, inv_s, cpar, true);
-    if (e0 + 3 < V) a += elem_weight(zv.w, qv.w, wm, fs, invtau, inv_s, cpar, true);
-    a = warp_sum(a);
-    if (lane == 0) seg_out[s] = a;
-    tot += a;
+  for (int base = warp; base < nloc; base += kAcceptWarps * kUnroll) {
+    float4 zv[kUnroll], qv[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int s = base + u * kAcceptWarps;
+      const int e0 = (seg0 + s) * kSeg + lane * 4;
+      if (s < nloc) {
+        zv[u] = load4(zr, e0, V, zvec, -INFINITY);
+        qv[u] = load4(qr, e0, V, qvec, 0.f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int s = base + u * kAcceptWarps;
+      if (s >= nloc) break;
+      const int e0 = (seg0 + s) * kSeg + lane * 4;
+      const float wm = sh.seg_m[s];
+      const double fs = sh.seg_f[s];
+      double a = 0.0;
+      if (e0 + 0 < V) a += elem_weight(zv[u].x, qv[u].x, wm, fs, invtau, inv_s, cpar, true);
+      if (e0 + 1 < V) a += elem_weight(zv[u].y, qv[u].y, wm, fs, invtau, inv_s, cpar, true);
+      if (e0 + 2 < V) a += elem_weight(zv[u].z, qv[u].z, wm, fs, invtau, inv_s, cpar, true);
+      if (e0 + 3 < V) a += elem_weight(zv[u].w, qv[u].w, wm, fs, invtau, inv_s, cpar, true);
+      a = warp_sum(a);
+      if (lane == 0) seg_out[s] = a;
+      tot += a;
+    }
   }
-  return block_sum_d(lane == 0 ? tot : 0.0, sh);
+  return block_sum_d(lane == 0 ? tot : 0.0, shw);
+}
+
+// Inverse-CDF search inside this CTA's slice: the first element where the
+// running sum (starting at `base`) exceeds `target`.  Run by warp 0 only;
+// returns t (or the slice's last positive element when rounding leaves the
+// crossing past the end) and the relative margin.
+__device__ void slice_search(const float* zr, const float* qr, bool zvec, bool qvec, int V, int seg0, int nloc,
+                             const AcceptShared& sh, const double* seg_w, double invtau, double inv_s,
+                             double cpar, bool resid, double base, double target, double W, int* out_t,
+                             double* out_margin) {
+  const int lane = threadIdx.x & 31;
+  const int per = (nloc + 31) / 32;
+  const int lo = min(lane * per, nloc), hi = min(lo + per, nloc);
+  double ls = 0.0;
+  for (int s = lo; s < hi; ++s) ls += seg_w[s];
+  const double incl = base + warp_incl_scan(ls);
+  double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) excl = base;
+  const unsigned m = __ballot_sync(0xffffffffu, incl > target);
+  int seg = -1;
+  double cb = 0.0;
+  bool found = false;
+  if (m != 0u) {
+    const int L = __ffs(m) - 1;
+    if (lane == L) {
+      double cum = excl;
+      int s = lo;
+      for (; s < hi; ++s) {
+        if (cum + seg_w[s] > target) break;
+        cum += seg_w[s];
+      }
+      seg = (s < hi) ? s : hi - 1;
+      cb = (s < hi) ? cum : cum - seg_w[hi - 1];
+    }
+    seg = __shfl_sync(0xffffffffu, seg, L);
+    cb = __shfl_sync(0xffffffffu, cb, L);
+    found = true;
+  } else {
+    int last = -1;
+    for (int s = lo; s < hi; ++s) if (seg_w[s] > 0.0) last = s;
+    const unsigned mm = __ballot_sync(0xffffffffu, last >= 0);
+    const int L = mm ? 31 - __clz(mm) : 0;
+    seg = __shfl_sync(0xffffffffu, last, L);
+    if (seg < 0) seg = 0;
+  }
+  const int e0 = (seg0 + seg) * kSeg + lane * 4;
+  const float4 zv = load4(zr, e0, V, zvec, -INFINITY);
+  float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (resid) qv = load4(qr, e0, V, qvec, 0.f);
+  const float wm = sh.seg_m[seg];
+  const double fs = sh.seg_f[seg];
+  double w[4];
+  w[0] = (e0 + 0 < V) ? elem_weight(zv.x, qv.x, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
+  w[1] = (e0 + 1 < V) ? elem_weight(zv.y, qv.y, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
+  w[2] = (e0 + 2 < V) ? elem_weight(zv.z, qv.z, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
+  w[3] = (e0 + 3 < V) ? elem_weight(zv.w, qv.w, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
+  int t = -1;
+  double margin = 0.0;
+  if (found) {
+    const double lsum = ((w[0] + w[1]) + w[2]) + w[3];
+    const double li = cb + warp_incl_scan(lsum);
+    double le = __shfl_up_sync(0xffffffffu, li, 1);
+    if (lane == 0) le = cb;
+    const unsigned m2 = __ballot_sync(0xffffffffu, li > target);
+    if (m2 != 0u) {
+      const int L = __ffs(m2) - 1;
+      if (lane == L) {
+        double cum = le;
+        for (int k = 0; k < 4; ++k) {
+          if (cum + w[k] > target) {
+            t = e0 + k;
+            margin = fmin(cum + w[k] - target, target - cum) / W;
+            break;
+          }
+          cum += w[k];
+        }
+      }
+      t = __shfl_sync(0xffffffffu, t, L);
+      margin = __shfl_sync(0xffffffffu, margin, L);
+    }
+  }
+  if (t < 0) {
+    int lp = -1;
+    for (int k = 0; k < 4; ++k) if (w[k] > 0.0) lp = e0 + k;
+    const unsigned mm = __ballot_sync(0xffffffffu, lp >= 0);
+    const int L = mm ? 31 - __clz(mm) : 0;
+    t = __shfl_sync(0xffffffffu, lp, L);
+    margin = 0.0;
+  }
+  *out_t = t;
+  *out_margin = margin;
+}
+
+// ------------------------------------------------------------ the walk
+
+// Called by every thread of one CTA: thread 0 follows the accepted children
+// from the root, then the block pads the outputs with -1.
+__device__ void accept_walk(const AcceptParams& p, int b, int n, AcceptShared& sh) {
+  const int T = p.T;
+  int32_t* acc = p.acc_nodes + static_cast<int64_t>(b) * T;
+  int32_t* out = p.out_tokens + static_cast<int64_t>(b) * (T + 1);
+  const int32_t* tok = p.tok + b * p.tok_sb;
+  const bool walk = (n > 0 && n <= T);
+  if (threadIdx.x == 0) {
+    int len = 0;
+    double mg = INFINITY;
+    if (walk) {
+      int c = 0;
+      int bonus = -1;
+      for (int step = 0; step < n; ++step) {
+        const AcceptDec* dp = p.dec + static_cast<int64_t>(b) * T + c;
+        const int child = __ldcg(&dp->child);
+        const int token = __ldcg(&dp->token);
+        mg = fmin(mg, __ldcg(&dp->margin));
+        if (child >= 0 && child < n) {
+          acc[len] = child;
+          out[len] = tok[child];
+          ++len;
+          c = child;
+        } else {
+          bonus = token;
+          if (bonus == kNonFiniteRow) {
+            set_status(p.status, TV_DEV_NONFINITE);
+            bonus = -1;
+          }
+          break;
+        }
+      }
+      out[len] = bonus;
+    }
+    p.n_acc[b] = len;
+    if (p.min_margin) p.min_margin[b] = mg;
+    sh.bc_int[1] = len;
+  }
+  __syncthreads();
+  const int len = sh.bc_int[1];
+  for (int i = len + threadIdx.x; i < T; i += blockDim.x) acc[i] = -1;
+  for (int i = len + (walk ? 1 : 0) + threadIdx.x; i < T + 1; i += blockDim.x) out[i] = -1;
 }
 
 // ------------------------------------------------------------ node kernel
 
-__global__ void __launch_bounds__(kAcceptThreads)
+__global__ void __launch_bounds__(kAcceptThreads, 2)
 accept_node_kernel(AcceptParams p) {
-  extern __shared__ double dyn_smem[];
   __shared__ AcceptShared sh;
-  const int c = blockIdx.x, b = blockIdx.y;
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = p.C;
+  const int rank = static_cast<int>(cl.block_rank());
+  const int c = blockIdx.x / C, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = p.n_nodes ? p.n_nodes[b] : p.T;
-  if (n < 0 || n > p.T) {
-    if (c == 0 && tid == 0) set_status(p.status, TV_DEV_BAD_LEN);
-    return;
+  if (n <= 0 || n > p.T) {
+    // nothing to decide: the first CTA writes the empty result
+    if (c == 0 && rank == 0) {
+      if (n != 0 && tid == 0) set_status(p.status, TV_DEV_BAD_LEN);
+      accept_walk(p, b, n, sh);
+    }
+    return;                                  // the whole cluster leaves together
   }
   if (c >= n) return;
   const int32_t* par = p.parent + b * p.par_sb;
   const int32_t* tok = p.tok + b * p.tok_sb;
-  if (tid == 0) {
+  if (rank == 0 && tid == 0) {
     uint32_t bits = 0;
     const int pc = par[c];
     if (c == 0 ? (pc != -1) : (pc < 0 || pc >= c)) bits |= TV_DEV_BAD_PARENT;
@@ -293,8 +371,12 @@ accept_node_kernel(AcceptParams p) {
   }
   const int V = p.V;
   const int nseg = (V + kSeg - 1) / kSeg;
+  const int seg0 = min(rank * p.seg_per_cta, nseg);
+  const int nloc = min(p.seg_per_cta, nseg - seg0);
   const float* zr = p.z + b * p.z_sb + c * p.z_st;
   const bool zvec = (reinterpret_cast<uintptr_t>(zr) & 15u) == 0;
+  int kred = 0;
+  Slot all[8];
   AcceptDec d;
   d.child = -1; d.token = -1; d.margin = INFINITY;
 
@@ -302,21 +384,30 @@ accept_node_kernel(AcceptParams p) {
     float bv = -INFINITY;
     int bi = INT_MAX;
     bool nan = false;
-    for (int s = warp; s < nseg; s += kAcceptWarps) {
-      const int e0 = s * kSeg + lane * 4;
-      const float4 v = load4(zr, e0, V, zvec, -INFINITY);
-      const float xs[4] = {v.x, v.y, v.z, v.w};
+    for (int base = warp; base < nloc; base += kAcceptWarps * kUnroll) {
+      float4 v[kUnroll];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int idx = e0 + k;
-        if (idx < V) {
-          const float x = xs[k];
-          if (isnan(x)) nan = true;
-          else if (x > bv || (x == bv && idx < bi)) { bv = x; bi = idx; }
+      for (int u = 0; u < kUnroll; ++u) {
+        const int s = base + u * kAcceptWarps;
+        if (s < nloc) v[u] = load4(zr, (seg0 + s) * kSeg + lane * 4, V, zvec, -INFINITY);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int s = base + u * kAcceptWarps;
+        if (s >= nloc) break;
+        const int e0 = (seg0 + s) * kSeg + lane * 4;
+        const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int idx = e0 + k;
+          if (idx < V) {
+            const float x = xs[k];
+            if (isnan(x)) nan = true;
+            else if (x > bv || (x == bv && idx < bi)) { bv = x; bi = idx; }
+          }
         }
       }
     }
-    // block argmax, ties to the lower index
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -326,22 +417,25 @@ accept_node_kernel(AcceptParams p) {
     const int any_nan = __syncthreads_or(nan ? 1 : 0);
     if (lane == 0) { sh.red_f[warp] = bv; sh.red_i[warp] = bi; }
     __syncthreads();
-    if (warp == 0) {
-      bv = (lane < kAcceptWarps) ? sh.red_f[lane] : -INFINITY;
-      bi = (lane < kAcceptWarps) ? sh.red_i[lane] : INT_MAX;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-      }
-      if (lane == 0) sh.bc_int[2] = bi;
+    Slot mine;
+    mine.a = 0.0; mine.b = 0.0; mine.f = -INFINITY; mine.i = INT_MAX; mine.j = any_nan;
+    if (tid == 0) {
+      float v = -INFINITY;
+      int i = INT_MAX;
+      for (int w = 0; w < kAcceptWarps; ++w)
+        if (sh.red_f[w] > v || (sh.red_f[w] == v && sh.red_i[w] < i)) { v = sh.red_f[w]; i = sh.red_i[w]; }
+      mine.f = v; mine.i = i;
     }
-    __syncthreads();
-    const int a = sh.bc_int[2];
-    if (any_nan) {
+    cluster_gather(cl, sh, mine, C, kred, all);
+    float gv = -INFINITY;
+    int a = INT_MAX, gnan = 0;
+    for (int r = 0; r < C; ++r) {
+      gnan |= all[r].j;
+      if (all[r].f > gv || (all[r].f == gv && all[r].i < a)) { gv = all[r].f; a = all[r].i; }
+    }
+    if (gnan) {
       d.token = kNonFiniteRow;
-    } else {
+    } else if (rank == 0) {
       d.child = first_child_with_token(par, tok, c, n, a, sh);
       d.token = (d.child >= 0) ? -1 : a;
     }
@@ -356,58 +450,89 @@ accept_node_kernel(AcceptParams p) {
     const bool read_q = specsample && has_child;
     const float* qr = read_q ? p.q + b * p.q_sb + c * p.q_st : nullptr;
     const bool qvec = read_q && ((reinterpret_cast<uintptr_t>(qr) & 15u) == 0);
-    // dynamic shared memory: seg_f, seg_w, seg_r (double) then seg_m (float)
-    double* seg_f = dyn_smem;
-    double* seg_w = seg_f + nseg;
-    double* seg_r = seg_w + nseg;
-    float* seg_m = reinterpret_cast<float*>(seg_r + nseg);
+    double* seg_w = sh.seg_w;
+    double* seg_r = sh.seg_r;
     const double invtau = 1.0 / static_cast<double>(p.tau);
 
     // pass 1: segment maxima and segment-frame exponential sums
     bool bad = false, qbad = false;
     float lmax = -INFINITY;
-    for (int s = warp; s < nseg; s += kAcceptWarps) {
-      const int e0 = s * kSeg + lane * 4;
-      const float4 v = load4(zr, e0, V, zvec, -INFINITY);
-      const float xs[4] = {v.x, v.y, v.z, v.w};
-      float m4 = -INFINITY;
+    for (int base = warp; base < nloc; base += kAcceptWarps * kUnroll) {
+      float4 v[kUnroll], qv[kUnroll];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (e0 + k < V) {
-          if (!isfinite(xs[k])) bad = true;
-          else m4 = fmaxf(m4, xs[k]);
+      for (int u = 0; u < kUnroll; ++u) {
+        const int s = base + u * kAcceptWarps;
+        if (s < nloc) {
+          const int e0 = (seg0 + s) * kSeg + lane * 4;
+          v[u] = load4(zr, e0, V, zvec, -INFINITY);
+          if (read_q) qv[u] = load4(qr, e0, V, qvec, 0.f);
         }
-      if (read_q) {
-        const float4 qv = load4(qr, e0, V, qvec, 0.f);
-        const float qs[4] = {qv.x, qv.y, qv.z, qv.w};
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int s = base + u * kAcceptWarps;
+        if (s >= nloc) break;
+        const int e0 = (seg0 + s) * kSeg + lane * 4;
+        const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        float m4 = -INFINITY;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          if (e0 + k < V && !(qs[k] >= 0.f && isfinite(qs[k]))) qbad = true;
-      }
-      const float wm = warp_max(m4);
-      double a = 0.0;
+          if (e0 + k < V) {
+            if (!isfinite(xs[k])) bad = true;
+            else m4 = fmaxf(m4, xs[k]);
+          }
+        if (read_q) {
+          const float qs[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (e0 + k < V && isfinite(xs[k]))
-          a += exp_neg((static_cast<double>(xs[k]) - static_cast<double>(wm)) * invtau);
-      a = warp_sum(a);
-      if (lane == 0) { seg_m[s] = wm; seg_w[s] = a; }
-      lmax = fmaxf(lmax, wm);
+          for (int k = 0; k < 4; ++k)
+            if (e0 + k < V && !(qs[k] >= 0.f && isfinite(qs[k]))) qbad = true;
+        }
+        const float wm = warp_max(m4);
+        double a = 0.0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (e0 + k < V && isfinite(xs[k]))
+            a += exp_neg((static_cast<double>(xs[k]) - static_cast<double>(wm)) * invtau);
+        a = warp_sum(a);
+        if (lane == 0) { sh.seg_m[s] = wm; seg_w[s] = a; }
+        lmax = fmaxf(lmax, wm);
+      }
     }
-    const int any_bad = __syncthreads_or(bad ? 1 : 0);
-    const int any_qbad = __syncthreads_or(qbad ? 1 : 0);
-    const float M = block_max_f(lmax, sh);
-    if (any_bad || any_qbad) {
+    const int any_bad = __syncthreads_or((bad || qbad) ? 1 : 0);
+    lmax = warp_max(lmax);
+    if (lane == 0) sh.red_f[warp] = lmax;
+    __syncthreads();
+    float cmax = -INFINITY;
+    for (int w = 0; w < kAcceptWarps; ++w) cmax = fmaxf(cmax, sh.red_f[w]);
+    // this CTA's sum in the frame of its own maximum
+    double part = 0.0;
+    for (int s = tid; s < nloc; s += blockDim.x)
+      part += seg_w[s] * exp((static_cast<double>(sh.seg_m[s]) - static_cast<double>(cmax)) * invtau);
+    const double csum = block_sum_d(part, sh);
+    Slot mine;
+    mine.a = csum; mine.b = 0.0; mine.f = cmax; mine.i = 0; mine.j = any_bad;
+    cluster_gather(cl, sh, mine, C, kred, all);
+    float M = -INFINITY;
+    int gbad = 0;
+    for (int r = 0; r < C; ++r) { M = fmaxf(M, all[r].f); gbad |= all[r].j; }
+    if (gbad) {
       d.token = kNonFiniteRow;
     } else {
-      double part = 0.0;
-      for (int s = tid; s < nseg; s += blockDim.x) {
-        const double f = exp((static_cast<double>(seg_m[s]) - static_cast<double>(M)) * invtau);
-        seg_f[s] = f;
+      double ssum = 0.0;
+      for (int r = 0; r < C; ++r)
+        if (all[r].f > -INFINITY)
+          ssum += all[r].a * exp((static_cast<double>(all[r].f) - static_cast<double>(M)) * invtau);
+      for (int s = tid; s < nloc; s += blockDim.x) {
+        const double f = exp((static_cast<double>(sh.seg_m[s]) - static_cast<double>(M)) * invtau);
+        sh.seg_f[s] = f;
         seg_w[s] *= f;
-        part += seg_w[s];
       }
-      const double ssum = block_sum_d(part, sh);   // syncs: seg_f / seg_w visible
+      // slice totals of the unnormalised softmax in the row frame
+      for (int r = 0; r < C; ++r)
+        sh.rank_tot[r] = (all[r].f > -INFINITY)
+                             ? all[r].a * exp((static_cast<double>(all[r].f) - static_cast<double>(M)) * invtau)
+                             : 0.0;
+      __syncthreads();
       const double inv_s = 1.0 / ssum;
       double margin = INFINITY;
       bool decided = false;
@@ -441,10 +566,8 @@ accept_node_kernel(AcceptParams p) {
             const int jc = sh.clist[ci];
             const int x = tok[jc];
             if (x < 0 || x >= V) continue;
-            // point value of the current distribution at x
-            const int sx = x / kSeg;
-            const double ex = exp_neg((static_cast<double>(zr[x]) - static_cast<double>(seg_m[sx])) * invtau) * seg_f[sx];
-            const double px = ex * inv_s;
+            // point value of the current distribution at x, in the row frame
+            const double px = exp((static_cast<double>(zr[x]) - static_cast<double>(M)) * invtau) * inv_s;
             const double qx = static_cast<double>(q[x]);
             const double num = px - cpar * qx;
             const double rx = num > 0.0 ? num / D : 0.0;
@@ -457,26 +580,58 @@ accept_node_kernel(AcceptParams p) {
               break;
             }
             const double cn = cpar + D;
-            const double S = residual_pass(zr, q, zvec, qvec, V, nseg, seg_m, seg_f, seg_r,
-                                           invtau, inv_s, cn, sh);
+            const double S_loc = residual_pass(zr, q, zvec, qvec, V, seg0, nloc, sh, seg_r, invtau, inv_s, cn, sh);
+            Slot ms;
+            ms.a = S_loc; ms.b = 0.0; ms.f = 0.f; ms.i = 0; ms.j = 0;
+            cluster_gather(cl, sh, ms, C, kred, all);
+            double S = 0.0;
+            for (int r = 0; r < C; ++r) S += all[r].a;
             if (S > 0.0) {
               cpar = cn; D = S; resid = true;
               double* t = seg_w; seg_w = seg_r; seg_r = t;
+              for (int r = 0; r < C; ++r) sh.rank_tot[r] = all[r].a;
             }
+            __syncthreads();
           }
         }
       }
       if (!decided) {
-        int t = -1;
-        double mg = 0.0;
+        // inverse-CDF sample over the current weights: find the CTA whose
+        // slice holds the crossing, search inside it, gather the result
         const int tag = specsample ? kTagResidual : kTagSpecExec;
         const double u = accept_uniform(p.seed, p.step, b, c, 0, tag);
-        sample_row(zr, qr, zvec, qvec, V, nseg, seg_m, seg_f, seg_w, invtau, inv_s, cpar,
-                   resid, u, &t, &mg, sh);
-        margin = fmin(margin, mg);
+        double W = 0.0;
+        for (int r = 0; r < C; ++r) W += sh.rank_tot[r];
+        const double target = u * W;
+        int owner = -1, last_pos = -1;
+        double base = 0.0, cum = 0.0;
+        for (int r = 0; r < C; ++r) {
+          if (sh.rank_tot[r] > 0.0) last_pos = r;
+          if (owner < 0 && cum + sh.rank_tot[r] > target) { owner = r; base = cum; }
+          if (owner < 0) cum += sh.rank_tot[r];
+        }
+        if (owner < 0) {                       // rounding: the last slice with weight
+          owner = last_pos < 0 ? 0 : last_pos;
+          base = 0.0;
+          for (int r = 0; r < owner; ++r) base += sh.rank_tot[r];
+        }
+        Slot res;
+        res.a = 0.0; res.b = 0.0; res.f = 0.f; res.i = -1; res.j = 0;
+        if (rank == owner && warp == 0) {
+          int t;
+          double mg;
+          slice_search(zr, qr, zvec, qvec, V, seg0, nloc, sh, seg_w, invtau, inv_s, cpar, resid, base,
+                       target, W, &t, &mg);
+          if (lane == 0) { sh.bc_int[2] = t; sh.bc_dbl[2] = mg; }
+        }
+        __syncthreads();
+        if (rank == owner) { res.i = sh.bc_int[2]; res.b = sh.bc_dbl[2]; }
+        cluster_gather(cl, sh, res, C, kred, all);
+        const int t = all[owner].i;
+        margin = fmin(margin, all[owner].b);
         if (specsample) {
           d.token = t;
-        } else {
+        } else if (rank == 0) {
           d.child = first_child_with_token(par, tok, c, n, t, sh);
           d.token = (d.child >= 0) ? -1 : t;
         }
@@ -484,57 +639,29 @@ accept_node_kernel(AcceptParams p) {
       d.margin = margin;
     }
   }
-  if (tid == 0) p.dec[static_cast<int64_t>(b) * p.T + c] = d;
-}
-
-// ------------------------------------------------------------ walk kernel
-
-__global__ void accept_walk_kernel(AcceptParams p) {
-  const int b = blockIdx.x;
-  const int lane = threadIdx.x;
-  const int T = p.T;
-  const int n = p.n_nodes ? p.n_nodes[b] : T;
-  int32_t* acc = p.acc_nodes + static_cast<int64_t>(b) * T;
-  int32_t* out = p.out_tokens + static_cast<int64_t>(b) * (T + 1);
-  const int32_t* tok = p.tok + b * p.tok_sb;
-  int len = 0;
-  double mg = INFINITY;
-  if (lane == 0 && n > 0 && n <= T) {
-    int c = 0;
-    int bonus = -1;
-    for (int step = 0; step < n; ++step) {
-      const AcceptDec d = p.dec[static_cast<int64_t>(b) * T + c];
-      mg = fmin(mg, d.margin);
-      if (d.child >= 0 && d.child < n) {
-        acc[len] = d.child;
-        out[len] = tok[d.child];
-        ++len;
-        c = d.child;
-      } else {
-        bonus = d.token;
-        if (bonus == kNonFiniteRow) {
-          set_status(p.status, TV_DEV_NONFINITE);
-          bonus = -1;
-        }
-        break;
-      }
+  // rank 0 publishes the decision; the last node of the sequence walks
+  if (rank == 0) {
+    if (tid == 0) {
+      p.dec[static_cast<int64_t>(b) * p.T + c] = d;
+      __threadfence();
+      const int done = atomicAdd(&p.ticket[b], 1);
+      sh.bc_int[2] = (done == n - 1);
     }
-    out[len] = bonus;
+    __syncthreads();
+    if (sh.bc_int[2]) {
+      __threadfence();
+      accept_walk(p, b, n, sh);
+      if (tid == 0) p.ticket[b] = 0;           // ready for the next call
+    }
   }
-  len = __shfl_sync(0xffffffffu, len, 0);
-  const bool wrote_bonus = (n > 0 && n <= T);
-  for (int i = len + lane; i < T; i += 32) acc[i] = -1;
-  for (int i = len + (wrote_bonus ? 1 : 0) + lane; i < T + 1; i += 32) out[i] = -1;
-  if (lane == 0) {
-    p.n_acc[b] = len;
-    if (p.min_margin) p.min_margin[b] = mg;
-  }
+  cl.sync();                                   // no CTA leaves while others may read its slots
 }
 
 // ------------------------------------------------------------ host side
 
 size_t accept_workspace_bytes(int B, int T) {
-  return static_cast<size_t>(B) * static_cast<size_t>(T) * sizeof(AcceptDec);
+  const size_t dec = static_cast<size_t>(B) * static_cast<size_t>(T) * sizeof(AcceptDec);
+  return ((dec + 255) & ~static_cast<size_t>(255)) + static_cast<size_t>(B) * sizeof(int32_t);
 }
 
 cudaError_t launch_accept(const tv_accept_args* a, int mode, void* ws, cudaStream_t stream) {
@@ -549,22 +676,34 @@ cudaError_t launch_accept(const tv_accept_args* a, int mode, void* ws, cudaStrea
   p.tau = a->temperature;
   p.seed = a->seed; p.step = a->step;
   p.status = a->dev_status;
+  const size_t dec = static_cast<size_t>(a->B) * static_cast<size_t>(a->T) * sizeof(AcceptDec);
   p.dec = static_cast<AcceptDec*>(ws);
+  p.ticket = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(ws) + ((dec + 255) & ~static_cast<size_t>(255)));
   p.n_acc = a->n_accepted; p.acc_nodes = a->accepted_nodes; p.out_tokens = a->out_tokens;
   p.min_margin = a->min_margin;
   if (a->B == 0) return cudaSuccess;
-  if (a->T > 0) {
-    const int nseg = (a->V + kSeg - 1) / kSeg;
-    const size_t smem = (mode == TV_ACCEPT_GREEDY) ? 0 : static_cast<size_t>(nseg) * (3 * sizeof(double) + sizeof(float));
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(accept_node_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-    }
-    dim3 grid(a->T, a->B);
-    accept_node_kernel<<<grid, kAcceptThreads, smem, stream>>>(p);
-  }
-  accept_walk_kernel<<<a->B, 32, 0, stream>>>(p);
+  const int nseg = (a->V + kSeg - 1) / kSeg;
+  int C = (nseg + 127) / 128;                  // ~16k elements per CTA
+  if (C < 1) C = 1;
+  if (C > 8) C = 8;
+  p.C = C;
+  p.seg_per_cta = (nseg + C - 1) / C;
+  if (p.seg_per_cta > kMaxSegPerCta) return cudaErrorInvalidValue;
+  const int rows = a->T > 0 ? a->T : 1;        // T == 0: one cluster writes the empty result
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows * C, a->B, 1);
+  cfg.blockDim = dim3(kAcceptThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, accept_node_kernel, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
