@@ -335,6 +335,12 @@ __device__ void accept_walk(const AcceptParams& p, int b, int n, AcceptShared& s
   const int len = sh.bc_int[1];
   for (int i = len + threadIdx.x; i < T; i += blockDim.x) acc[i] = -1;
   for (int i = len + (walk ? 1 : 0) + threadIdx.x; i < T + 1; i += blockDim.x) out[i] = -1;
+  // leave the workspace zero: the next call may lay it out differently
+  if (walk) {
+    AcceptDec z;
+    z.child = 0; z.token = 0; z.margin = 0.0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) p.dec[static_cast<int64_t>(b) * T + i] = z;
+  }
 }
 
 // ------------------------------------------------------------ node kernel
