@@ -63,7 +63,7 @@ struct AcceptParams {
   int seg_per_cta;          // 128-element segments per CTA
 };
 
-constexpr int kAcceptThreads = 512;
+constexpr int kAcceptThreads = 256;
 constexpr int kAcceptWarps = kAcceptThreads / kWarp;
 constexpr int kSeg = 128;
 constexpr int kUnroll = 2;
@@ -141,14 +141,15 @@ __device__ __forceinline__ void cluster_gather(cg::cluster_group& cl, AcceptShar
   ++k;
 }
 
-// Weight of one element in the current distribution: e = exp((z-wm)/tau) *
-// f_seg (unnormalised softmax), or the residual (e/s - c q)^+.
-__device__ __forceinline__ double elem_weight(float z, float q, float wm, double fseg, double invtau,
-                                              double inv_s, double cpar, bool resid) {
-  const double e = exp_neg((static_cast<double>(z) - static_cast<double>(wm)) * invtau) * fseg;
+// Weight of one element in the current distribution, in fp32: with
+// e = exp((z - wm)/tau) in the segment frame, the unnormalised softmax
+// weight is e * fs (fs = f_seg) and the residual weight is
+// (e * fs - c q)^+ (fs = f_seg / s).  Sums are accumulated in fp64.
+__device__ __forceinline__ float elem_weight(float z, float q, float wm, float fs, float invtau, float cpar,
+                                             bool resid) {
+  const float e = expf((z - wm) * invtau) * fs;
   if (!resid) return e;
-  const double w = e * inv_s - cpar * static_cast<double>(q);
-  return w > 0.0 ? w : 0.0;
+  return fmaxf(fmaf(-cpar, q, e), 0.f);
 }
 
 // Lowest-index child of c (c < j < n) that carries token x, or -1.
@@ -164,9 +165,10 @@ __device__ int first_child_with_token(const int32_t* par, const int32_t* tok, in
 // One pass over this CTA's slice computing the segment sums of the residual
 // weights (e/s - c q)^+ into seg_out; returns the slice total.
 __device__ double residual_pass(const float* zr, const float* qr, bool zvec, bool qvec, int V, int seg0,
-                                int nloc, const AcceptShared& sh, double* seg_out, double invtau, double inv_s,
+                                int nloc, const AcceptShared& sh, double* seg_out, float invtau, double inv_s,
                                 double cpar, AcceptShared& shw) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float cf = static_cast<float>(cpar);
   double tot = 0.0;
   for (int base = warp; base < nloc; base += kAcceptWarps * kUnroll) {
     float4 zv[kUnroll], qv[kUnroll];
@@ -185,15 +187,15 @@ __device__ double residual_pass(const float* zr, const float* qr, bool zvec, boo
       if (s >= nloc) break;
       const int e0 = (seg0 + s) * kSeg + lane * 4;
       const float wm = sh.seg_m[s];
-      const double fs = sh.seg_f[s];
-      double a = 0.0;
-      if (e0 + 0 < V) a += elem_weight(zv[u].x, qv[u].x, wm, fs, invtau, inv_s, cpar, true);
-      if (e0 + 1 < V) a += elem_weight(zv[u].y, qv[u].y, wm, fs, invtau, inv_s, cpar, true);
-      if (e0 + 2 < V) a += elem_weight(zv[u].z, qv[u].z, wm, fs, invtau, inv_s, cpar, true);
-      if (e0 + 3 < V) a += elem_weight(zv[u].w, qv[u].w, wm, fs, invtau, inv_s, cpar, true);
-      a = warp_sum(a);
-      if (lane == 0) seg_out[s] = a;
-      tot += a;
+      const float fs = static_cast<float>(sh.seg_f[s] * inv_s);
+      float a = 0.f;
+      if (e0 + 0 < V) a += elem_weight(zv[u].x, qv[u].x, wm, fs, invtau, cf, true);
+      if (e0 + 1 < V) a += elem_weight(zv[u].y, qv[u].y, wm, fs, invtau, cf, true);
+      if (e0 + 2 < V) a += elem_weight(zv[u].z, qv[u].z, wm, fs, invtau, cf, true);
+      if (e0 + 3 < V) a += elem_weight(zv[u].w, qv[u].w, wm, fs, invtau, cf, true);
+      const double ad = warp_sum(static_cast<double>(a));
+      if (lane == 0) seg_out[s] = ad;
+      tot += ad;
     }
   }
   return block_sum_d(lane == 0 ? tot : 0.0, shw);
@@ -204,7 +206,7 @@ __device__ double residual_pass(const float* zr, const float* qr, bool zvec, boo
 // returns t (or the slice's last positive element when rounding leaves the
 // crossing past the end) and the relative margin.
 __device__ void slice_search(const float* zr, const float* qr, bool zvec, bool qvec, int V, int seg0, int nloc,
-                             const AcceptShared& sh, const double* seg_w, double invtau, double inv_s,
+                             const AcceptShared& sh, const double* seg_w, float invtau, double inv_s,
                              double cpar, bool resid, double base, double target, double W, int* out_t,
                              double* out_margin) {
   const int lane = threadIdx.x & 31;
@@ -247,12 +249,13 @@ __device__ void slice_search(const float* zr, const float* qr, bool zvec, bool q
   float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
   if (resid) qv = load4(qr, e0, V, qvec, 0.f);
   const float wm = sh.seg_m[seg];
-  const double fs = sh.seg_f[seg];
+  const float fs = static_cast<float>(resid ? sh.seg_f[seg] * inv_s : sh.seg_f[seg]);
+  const float cf = static_cast<float>(cpar);
   double w[4];
-  w[0] = (e0 + 0 < V) ? elem_weight(zv.x, qv.x, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
-  w[1] = (e0 + 1 < V) ? elem_weight(zv.y, qv.y, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
-  w[2] = (e0 + 2 < V) ? elem_weight(zv.z, qv.z, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
-  w[3] = (e0 + 3 < V) ? elem_weight(zv.w, qv.w, wm, fs, invtau, inv_s, cpar, resid) : 0.0;
+  w[0] = (e0 + 0 < V) ? static_cast<double>(elem_weight(zv.x, qv.x, wm, fs, invtau, cf, resid)) : 0.0;
+  w[1] = (e0 + 1 < V) ? static_cast<double>(elem_weight(zv.y, qv.y, wm, fs, invtau, cf, resid)) : 0.0;
+  w[2] = (e0 + 2 < V) ? static_cast<double>(elem_weight(zv.z, qv.z, wm, fs, invtau, cf, resid)) : 0.0;
+  w[3] = (e0 + 3 < V) ? static_cast<double>(elem_weight(zv.w, qv.w, wm, fs, invtau, cf, resid)) : 0.0;
   int t = -1;
   double margin = 0.0;
   if (found) {
@@ -345,7 +348,7 @@ __device__ void accept_walk(const AcceptParams& p, int b, int n, AcceptShared& s
 
 // ------------------------------------------------------------ node kernel
 
-__global__ void __launch_bounds__(kAcceptThreads, 2)
+__global__ void __launch_bounds__(kAcceptThreads, 4)
 accept_node_kernel(AcceptParams p) {
   __shared__ AcceptShared sh;
   cg::cluster_group cl = cg::this_cluster();
@@ -459,6 +462,7 @@ accept_node_kernel(AcceptParams p) {
     double* seg_w = sh.seg_w;
     double* seg_r = sh.seg_r;
     const double invtau = 1.0 / static_cast<double>(p.tau);
+    const float invtau_f = 1.0f / p.tau;
 
     // pass 1: segment maxima and segment-frame exponential sums
     bool bad = false, qbad = false;
@@ -494,12 +498,11 @@ accept_node_kernel(AcceptParams p) {
             if (e0 + k < V && !(qs[k] >= 0.f && isfinite(qs[k]))) qbad = true;
         }
         const float wm = warp_max(m4);
-        double a = 0.0;
+        float af = 0.f;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          if (e0 + k < V && isfinite(xs[k]))
-            a += exp_neg((static_cast<double>(xs[k]) - static_cast<double>(wm)) * invtau);
-        a = warp_sum(a);
+          if (e0 + k < V && isfinite(xs[k])) af += expf((xs[k] - wm) * invtau_f);
+        const double a = warp_sum(static_cast<double>(af));
         if (lane == 0) { sh.seg_m[s] = wm; seg_w[s] = a; }
         lmax = fmaxf(lmax, wm);
       }
@@ -586,7 +589,7 @@ accept_node_kernel(AcceptParams p) {
               break;
             }
             const double cn = cpar + D;
-            const double S_loc = residual_pass(zr, q, zvec, qvec, V, seg0, nloc, sh, seg_r, invtau, inv_s, cn, sh);
+            const double S_loc = residual_pass(zr, q, zvec, qvec, V, seg0, nloc, sh, seg_r, invtau_f, inv_s, cn, sh);
             Slot ms;
             ms.a = S_loc; ms.b = 0.0; ms.f = 0.f; ms.i = 0; ms.j = 0;
             cluster_gather(cl, sh, ms, C, kred, all);
@@ -626,7 +629,7 @@ accept_node_kernel(AcceptParams p) {
         if (rank == owner && warp == 0) {
           int t;
           double mg;
-          slice_search(zr, qr, zvec, qvec, V, seg0, nloc, sh, seg_w, invtau, inv_s, cpar, resid, base,
+          slice_search(zr, qr, zvec, qvec, V, seg0, nloc, sh, seg_w, invtau_f, inv_s, cpar, resid, base,
                        target, W, &t, &mg);
           if (lane == 0) { sh.bc_int[2] = t; sh.bc_dbl[2] = mg; }
         }

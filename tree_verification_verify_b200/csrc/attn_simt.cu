@@ -135,11 +135,14 @@ attn_prefix_simt_kernel(AttnParams p) {
 
 constexpr int kTreeThreads = 128;
 constexpr int kTreeWarps = kTreeThreads / kWarp;
+constexpr int kTreeStage = 32;                    // path rows staged per round
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kTreeThreads)
 attn_tree_kernel(AttnParams p) {
   extern __shared__ int path_smem[];              // [T] ancestor list
+  __shared__ float ks[kTreeStage][D];
+  __shared__ float vs[kTreeStage][D];
   __shared__ int s_len, s_ok;
   constexpr int DL = D / 32;
   const int i = blockIdx.x;
@@ -164,40 +167,62 @@ attn_tree_kernel(AttnParams p) {
     if (g == 0) p.node_ok[static_cast<int64_t>(b) * p.T + i] = ok;
   }
   __syncthreads();
-  const int len = s_len;
-  const int ok = s_ok;
+  const int len = s_ok ? s_len : 0;
   const int G = p.G;
-  for (int hg = warp; hg < G; hg += kTreeWarps) {
-    const int h = g * G + hg;
-    float qv[DL], acc[DL];
+  float qv[kTreeWarps > 0 ? 8 : 1][DL];            // up to 8 heads per warp
+  float acc[8][DL], m[8], l[8];
+  const int nh = (G + kTreeWarps - 1) / kTreeWarps;   // heads per warp (<= 16 for G <= 64)
+  for (int h0 = 0; h0 < nh; h0 += 8) {
 #pragma unroll
-    for (int k = 0; k < DL; ++k) {
-      qv[k] = ld_elt<T>(p.q, b * p.q_sb + i * p.q_st + h * p.q_sh + lane + 32 * k) * p.scale;
-      acc[k] = 0.f;
-    }
-    float m = -INFINITY, l = 0.f;
-    if (ok) {
-      for (int t = 0; t < len; ++t) {
-        const int j = path_smem[t];
-        const int64_t off = b * p.kt_sb + static_cast<int64_t>(j) * p.kt_st + g * p.kt_sh;
-        float s = 0.f;
+    for (int r = 0; r < 8; ++r) {
+      const int hg = warp + (h0 + r) * kTreeWarps;
+      m[r] = -INFINITY; l[r] = 0.f;
 #pragma unroll
-        for (int k = 0; k < DL; ++k) s = fmaf(qv[k], ld_elt<T>(p.kt, off + lane + 32 * k), s);
-        s = warp_sumf(s);
-        const float mn = fmaxf(m, s);
-        const float corr = expf(m - mn);
-        const float pj = expf(s - mn);
-        l = l * corr + pj;
-#pragma unroll
-        for (int k = 0; k < DL; ++k) acc[k] = fmaf(pj, ld_elt<T>(p.vt, off + lane + 32 * k), acc[k] * corr);
-        m = mn;
+      for (int k = 0; k < DL; ++k) {
+        acc[r][k] = 0.f;
+        qv[r][k] = (hg < G) ? ld_elt<T>(p.q, b * p.q_sb + i * p.q_st + (g * G + hg) * p.q_sh + lane + 32 * k) * p.scale
+                            : 0.f;
       }
     }
-    const int64_t pr = part_row(p, p.nchunk, b, i, h);
-    const float inv = l > 0.f ? 1.f / l : 0.f;
+    for (int t0 = 0; t0 < len; t0 += kTreeStage) {
+      const int nt = min(kTreeStage, len - t0);
+      __syncthreads();
+      for (int e = threadIdx.x; e < nt * D; e += blockDim.x) {
+        const int t = e / D, dd = e % D;
+        const int64_t off = b * p.kt_sb + static_cast<int64_t>(path_smem[t0 + t]) * p.kt_st + g * p.kt_sh + dd;
+        ks[t][dd] = ld_elt<T>(p.kt, off);
+        vs[t][dd] = ld_elt<T>(p.vt, off);
+      }
+      __syncthreads();
 #pragma unroll
-    for (int k = 0; k < DL; ++k) p.part_o[pr * D + lane + 32 * k] = acc[k] * inv;
-    if (lane == 0) p.part_lse[pr] = l > 0.f ? m + logf(l) : -INFINITY;
+      for (int r = 0; r < 8; ++r) {
+        const int hg = warp + (h0 + r) * kTreeWarps;
+        if (hg >= G) break;
+        for (int t = 0; t < nt; ++t) {
+          float s = 0.f;
+#pragma unroll
+          for (int k = 0; k < DL; ++k) s = fmaf(qv[r][k], ks[t][lane + 32 * k], s);
+          s = warp_sumf(s);
+          const float mn = fmaxf(m[r], s);
+          const float corr = expf(m[r] - mn);
+          const float pj = expf(s - mn);
+          l[r] = l[r] * corr + pj;
+#pragma unroll
+          for (int k = 0; k < DL; ++k) acc[r][k] = fmaf(pj, vs[t][lane + 32 * k], acc[r][k] * corr);
+          m[r] = mn;
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int hg = warp + (h0 + r) * kTreeWarps;
+      if (hg >= G) break;
+      const int64_t pr = part_row(p, p.nchunk, b, i, g * G + hg);
+      const float inv = l[r] > 0.f ? 1.f / l[r] : 0.f;
+#pragma unroll
+      for (int k = 0; k < DL; ++k) p.part_o[pr * D + lane + 32 * k] = acc[r][k] * inv;
+      if (lane == 0) p.part_lse[pr] = l[r] > 0.f ? m[r] + logf(l[r]) : -INFINITY;
+    }
   }
 }
 
@@ -234,17 +259,20 @@ attn_merge_kernel(AttnParams p) {
     if (p.lse && lane == 0) p.lse[row] = NAN;
     return;
   }
-  float M = -INFINITY;
-  for (int c = 0; c <= p.nchunk; ++c) M = fmaxf(M, p.part_lse[part_row(p, c, b, i, h)]);
-  float den = 0.f, acc[DL];
+  // partial c's lse in lane c (at most 32 partials), weights by warp max
+  const int np = p.nchunk + 1;
+  float lc = -INFINITY;
+  for (int c = lane; c < np; c += 32) lc = fmaxf(lc, p.part_lse[part_row(p, c, b, i, h)]);
+  const float M = warp_max(lc);
+  float wl = (lane < np && lc > -INFINITY) ? expf(lc - M) : 0.f;
+  float den = warp_sumf(wl);
+  float acc[DL];
 #pragma unroll
   for (int k = 0; k < DL; ++k) acc[k] = 0.f;
-  for (int c = 0; c <= p.nchunk; ++c) {
+  for (int c = 0; c < np; ++c) {
+    const float w = __shfl_sync(0xffffffffu, wl, c & 31);
+    if (w == 0.f) continue;
     const int64_t pr = part_row(p, c, b, i, h);
-    const float lc = p.part_lse[pr];
-    if (lc == -INFINITY) continue;
-    const float w = expf(lc - M);
-    den += w;
 #pragma unroll
     for (int k = 0; k < DL; ++k) acc[k] = fmaf(w, p.part_o[pr * D + lane + 32 * k], acc[k]);
   }

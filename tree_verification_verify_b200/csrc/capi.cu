@@ -74,9 +74,15 @@ AttnPlan plan_attn(const tv_attn_args* a) {
     pl.nchunk = pl.sparse ? 1 : 0;
     pl.chunk_len = 128;
   } else {
-    const int64_t target = 3LL * num_sms();
+    // about four waves of CTAs (balance across ragged prefixes), but at least four 128-key tiles per
+    // chunk for the tensor-core kernel (its pipeline and the partial
+    // write-back are amortised over the chunk), and at most 31 chunks so
+    // that the merge reads every partial of a row with one warp
+    const int64_t target = 4LL * num_sms();
     int64_t want = (target + units - 1) / units;
-    const int64_t maxc = (a->Lmax + 127) / 128;
+    int64_t maxc = (a->Lmax + 127) / 128;
+    if (pl.tc) maxc = (a->Lmax + 511) / 512;
+    if (maxc > 31) maxc = 31;
     if (want < 1) want = 1;
     if (want > maxc) want = maxc;
     int64_t len = (a->Lmax + want - 1) / want;
