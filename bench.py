@@ -11,10 +11,13 @@ tree tokens per second per layer over all ranks.  Inputs are synthetic
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--config llama3_8b|specexec70b|serving|longctx|longctx_sparse]
 
-Timing: W untimed warm-up steps, then K steps, each preceded (outside the
-timed region) by a 256 MiB write that flushes the 126 MB L2; each step is
+Timing: the two calls of a step are captured once into CUDA graphs; W
+untimed warm-up steps, then K steps, each preceded (outside the timed
+region) by a 256 MiB write that flushes the 126 MB L2; each step is
 bracketed by CUDA events on the launching stream, per-call events give the
-per-call durations; the max over ranks is reported.  --impl reference times
+per-call durations; the max over ranks is reported.  The e2e figure calls
+the Python API directly (no graph), copying the step's inputs from pinned
+host memory and reading the accepted tokens back.  --impl reference times
 the fp64 CPU oracle on a bounded sample of the same workload.
 """
 
@@ -218,12 +221,33 @@ class Step:
         return (5 if self.sparse else 3) + 2
 
 
+def capture_graphs(step):
+    """CUDA graphs of the two calls of a step (captured once, replayed in
+    the timed region so that no host launch overhead sits between kernels)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):                       # warm the library's host-side setup
+            step.run_attn()
+            step.run_accept()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g_attn, g_acc = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_attn):
+        step.run_attn()
+    with torch.cuda.graph(g_acc):
+        step.run_accept()
+    torch.cuda.synchronize()
+    return g_attn, g_acc
+
+
 def time_steps(step, K, W, world, flush):
+    g_attn, g_acc = capture_graphs(step)
     s = torch.cuda.current_stream()
     for _ in range(W):
         flush.zero_()
-        step.run_attn()
-        step.run_accept()
+        g_attn.replay()
+        g_acc.replay()
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     barrier(world)
@@ -231,14 +255,15 @@ def time_steps(step, K, W, world, flush):
     for k in range(K):
         flush.zero_()
         ev[k][0].record(s)
-        step.run_attn()
+        g_attn.replay()
         ev[k][1].record(s)
-        step.run_accept()
+        g_acc.replay()
         ev[k][2].record(s)
     torch.cuda.synchronize()
     barrier(world)
     t_attn = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
     t_acc = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    del g_attn, g_acc
     return t_attn, t_acc
 
 
@@ -337,6 +362,7 @@ def config_block(step, world):
                         f"prefix={c['L']} T={c['T']} V={c['V']} temp={step.temperature}"
                         + (" sparse top-32 blocks of 64" if step.sparse else ""),
             "tree_nodes_per_rank": step.B * step.T, "l2": "256 MiB flush before every timed step (not timed)",
+            "launch": "each call replayed from a CUDA graph",
             "parallelism": f"replicas x{world}"}
 
 
