@@ -232,10 +232,12 @@ def capture_graphs(step):
             step.run_accept()
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
+    # capture on the warm-up stream: the binding's per-stream workspace then
+    # already exists and nothing is allocated (or zero-filled) in the graph
     g_attn, g_acc = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_attn):
+    with torch.cuda.graph(g_attn, stream=s):
         step.run_attn()
-    with torch.cuda.graph(g_acc):
+    with torch.cuda.graph(g_acc, stream=s):
         step.run_accept()
     torch.cuda.synchronize()
     return g_attn, g_acc
