@@ -15,17 +15,21 @@
 //
 // Layout of a row pass.  A thread-block cluster of C CTAs (C <= 8) owns one
 // node row; CTA rank r owns a contiguous slice of 128-element segments.  A
-// warp owns a segment (lane l holds elements 4l..4l+3, one 16-byte load) and
-// keeps four segments in flight.  Cross-CTA sums and maxima go through
-// distributed shared memory (double-buffered slots, one cluster barrier per
-// reduction); every CTA of the cluster computes the same reduced values and
-// so takes the same branches.
+// warp owns a segment at a time (lane l holds elements 4l..4l+3, one 16-byte
+// load) and keeps kUnroll segments in flight.  Cross-CTA sums and maxima go
+// through distributed shared memory (double-buffered slots, one cluster
+// barrier per reduction); every CTA computes the same reduced values and so
+// takes the same branches.
 //
-// Per segment the first pass keeps the segment maximum wm and the sum of
-// exp((z - wm)/tau); element weights are recomputed in that same segment
-// frame, scaled by f_seg = exp((wm - M)/tau) (M the row maximum).  Residuals
-// are parametrised as r = (p - c q)^+ / D: rejecting a child with the
-// current (c, D) gives c' = c + D and D' = sum_t (p - c' q)^+, one pass.
+// Arithmetic.  The row maximum M is found first; every element weight is
+// then e_t = 2^(z_t * k - M * k) with k = log2(e) / tau (one FFMA and one
+// ex2.approx), the unnormalised softmax.  Residuals are parametrised as
+// r = (p - c q)^+ / D with p = e / s: rejecting a child with the current
+// (c, D) gives c' = c + D and D' = sum_t (p_t - c' q_t)^+, one pass.
+// Weights are fp32; each lane's four weights are summed in fp32, segment
+// sums are fp32 warp reductions and everything above that is fp64.  The
+// segment sums are kept in shared memory, so an inverse-CDF sample re-reads
+// one segment only.
 #include <cooperative_groups.h>
 
 #include "tv_common.cuh"
@@ -66,7 +70,7 @@ struct AcceptParams {
 constexpr int kAcceptThreads = 256;
 constexpr int kAcceptWarps = kAcceptThreads / kWarp;
 constexpr int kSeg = 128;
-constexpr int kUnroll = 2;
+constexpr int kUnroll = 4;
 constexpr int kMaxSegPerCta = 512;      // 65536 elements per CTA
 
 // ------------------------------------------------------------ shared state
@@ -81,18 +85,34 @@ struct AcceptShared {
   double red_d[kAcceptWarps];
   float red_f[kAcceptWarps];
   int red_i[kAcceptWarps];
-  int red_j[kAcceptWarps];
   int wofs[kAcceptWarps];
   int clist[kAcceptThreads];
   int bc_int[4];
   double bc_dbl[4];
   Slot slot[2];
-  double rank_tot[8];      // per-CTA totals of the current weights
-  float seg_m[kMaxSegPerCta];
-  double seg_f[kMaxSegPerCta];
-  double seg_w[kMaxSegPerCta];
-  double seg_r[kMaxSegPerCta];
+  double rank_tot[8];           // per-CTA totals of the current weights
+  float seg_a[kMaxSegPerCta];   // segment sums of the current weights
+  float seg_b[kMaxSegPerCta];   // scratch for a residual pass
 };
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Element weight: e = 2^(z k + zoff) (zoff = -M k), or the residual
+// (e * inv_s - c q)^+.
+__device__ __forceinline__ float weight(float z, float q, float k, float zoff, float inv_s, float c, bool resid) {
+  const float e = ex2_approx(fmaf(z, k, zoff));
+  return resid ? fmaxf(fmaf(-c, q, e * inv_s), 0.f) : e;
+}
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
 
 __device__ __forceinline__ double block_sum_d(double v, AcceptShared& sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -100,13 +120,10 @@ __device__ __forceinline__ double block_sum_d(double v, AcceptShared& sh) {
   __syncthreads();
   if (lane == 0) sh.red_d[warp] = v;
   __syncthreads();
-  if (warp == 0) {
-    double t = (lane < kAcceptWarps) ? sh.red_d[lane] : 0.0;
-    t = warp_sum(t);
-    if (lane == 0) sh.bc_dbl[0] = t;
-  }
-  __syncthreads();
-  return sh.bc_dbl[0];
+  double t = 0.0;
+#pragma unroll
+  for (int w = 0; w < kAcceptWarps; ++w) t += sh.red_d[w];
+  return t;
 }
 
 __device__ __forceinline__ int block_min_i(int v, AcceptShared& sh) {
@@ -116,14 +133,10 @@ __device__ __forceinline__ int block_min_i(int v, AcceptShared& sh) {
   __syncthreads();
   if (lane == 0) sh.red_i[warp] = v;
   __syncthreads();
-  if (warp == 0) {
-    int t = (lane < kAcceptWarps) ? sh.red_i[lane] : INT_MAX;
+  int t = INT_MAX;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) t = min(t, __shfl_xor_sync(0xffffffffu, t, o));
-    if (lane == 0) sh.bc_int[0] = t;
-  }
-  __syncthreads();
-  return sh.bc_int[0];
+  for (int w = 0; w < kAcceptWarps; ++w) t = min(t, sh.red_i[w]);
+  return t;
 }
 
 // Cluster all-gather of one Slot per CTA: after the call every thread of
@@ -134,22 +147,8 @@ __device__ __forceinline__ void cluster_gather(cg::cluster_group& cl, AcceptShar
   Slot* s = &sh.slot[k & 1];
   if (threadIdx.x == 0) *s = mine;
   cl.sync();
-  for (int r = 0; r < C; ++r) {
-    const Slot* rs = cl.map_shared_rank(s, r);
-    out[r] = *rs;
-  }
+  for (int r = 0; r < C; ++r) out[r] = *cl.map_shared_rank(s, r);
   ++k;
-}
-
-// Weight of one element in the current distribution, in fp32: with
-// e = exp((z - wm)/tau) in the segment frame, the unnormalised softmax
-// weight is e * fs (fs = f_seg) and the residual weight is
-// (e * fs - c q)^+ (fs = f_seg / s).  Sums are accumulated in fp64.
-__device__ __forceinline__ float elem_weight(float z, float q, float wm, float fs, float invtau, float cpar,
-                                             bool resid) {
-  const float e = expf((z - wm) * invtau) * fs;
-  if (!resid) return e;
-  return fmaxf(fmaf(-cpar, q, e), 0.f);
 }
 
 // Lowest-index child of c (c < j < n) that carries token x, or -1.
@@ -162,58 +161,60 @@ __device__ int first_child_with_token(const int32_t* par, const int32_t* tok, in
   return best == INT_MAX ? -1 : best;
 }
 
-// One pass over this CTA's slice computing the segment sums of the residual
-// weights (e/s - c q)^+ into seg_out; returns the slice total.
-__device__ double residual_pass(const float* zr, const float* qr, bool zvec, bool qvec, int V, int seg0,
-                                int nloc, const AcceptShared& sh, double* seg_out, float invtau, double inv_s,
-                                double cpar, AcceptShared& shw) {
+struct Frame {
+  float k, zoff, inv_s, c;   // weight parameters
+  bool resid;
+};
+
+// One pass over this CTA's slice: segment sums of the current weights into
+// seg_out; returns the slice total (fp64).
+template <bool READQ>
+__device__ double weight_pass(const float* zr, const float* qr, bool zvec, bool qvec, int V, int seg0, int nloc,
+                              const Frame& f, float* seg_out, AcceptShared& sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const float cf = static_cast<float>(cpar);
   double tot = 0.0;
   for (int base = warp; base < nloc; base += kAcceptWarps * kUnroll) {
     float4 zv[kUnroll], qv[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int s = base + u * kAcceptWarps;
-      const int e0 = (seg0 + s) * kSeg + lane * 4;
       if (s < nloc) {
+        const int e0 = (seg0 + s) * kSeg + lane * 4;
         zv[u] = load4(zr, e0, V, zvec, -INFINITY);
-        qv[u] = load4(qr, e0, V, qvec, 0.f);
+        if (READQ) qv[u] = load4(qr, e0, V, qvec, 0.f);
+        else qv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int s = base + u * kAcceptWarps;
-      if (s >= nloc) break;
-      const int e0 = (seg0 + s) * kSeg + lane * 4;
-      const float wm = sh.seg_m[s];
-      const float fs = static_cast<float>(sh.seg_f[s] * inv_s);
-      float a = 0.f;
-      if (e0 + 0 < V) a += elem_weight(zv[u].x, qv[u].x, wm, fs, invtau, cf, true);
-      if (e0 + 1 < V) a += elem_weight(zv[u].y, qv[u].y, wm, fs, invtau, cf, true);
-      if (e0 + 2 < V) a += elem_weight(zv[u].z, qv[u].z, wm, fs, invtau, cf, true);
-      if (e0 + 3 < V) a += elem_weight(zv[u].w, qv[u].w, wm, fs, invtau, cf, true);
-      const double ad = warp_sum(static_cast<double>(a));
-      if (lane == 0) seg_out[s] = ad;
-      tot += ad;
+      if (s < nloc) {
+        // fill values (-inf logits) give weight 0 past the row end
+        float g = weight(zv[u].x, qv[u].x, f.k, f.zoff, f.inv_s, f.c, f.resid);
+        g += weight(zv[u].y, qv[u].y, f.k, f.zoff, f.inv_s, f.c, f.resid);
+        g += weight(zv[u].z, qv[u].z, f.k, f.zoff, f.inv_s, f.c, f.resid);
+        g += weight(zv[u].w, qv[u].w, f.k, f.zoff, f.inv_s, f.c, f.resid);
+        const float ss = warp_sum_f(g);
+        if (lane == 0) seg_out[s] = ss;
+        tot += static_cast<double>(ss);
+      }
     }
   }
-  return block_sum_d(lane == 0 ? tot : 0.0, shw);
+  return block_sum_d(lane == 0 ? tot : 0.0, sh);
 }
 
-// Inverse-CDF search inside this CTA's slice: the first element where the
-// running sum (starting at `base`) exceeds `target`.  Run by warp 0 only;
-// returns t (or the slice's last positive element when rounding leaves the
+// Inverse-CDF search inside this CTA's slice (run by warp 0): the first
+// element where the running sum, starting at `base`, exceeds `target`.
+// Returns t (or the slice's last positive element when rounding leaves the
 // crossing past the end) and the relative margin.
 __device__ void slice_search(const float* zr, const float* qr, bool zvec, bool qvec, int V, int seg0, int nloc,
-                             const AcceptShared& sh, const double* seg_w, float invtau, double inv_s,
-                             double cpar, bool resid, double base, double target, double W, int* out_t,
+                             const float* seg_w, const Frame& f, double base, double target, double W, int* out_t,
                              double* out_margin) {
   const int lane = threadIdx.x & 31;
   const int per = (nloc + 31) / 32;
   const int lo = min(lane * per, nloc), hi = min(lo + per, nloc);
   double ls = 0.0;
-  for (int s = lo; s < hi; ++s) ls += seg_w[s];
+  for (int s = lo; s < hi; ++s) ls += static_cast<double>(seg_w[s]);
   const double incl = base + warp_incl_scan(ls);
   double excl = __shfl_up_sync(0xffffffffu, incl, 1);
   if (lane == 0) excl = base;
@@ -227,18 +228,18 @@ __device__ void slice_search(const float* zr, const float* qr, bool zvec, bool q
       double cum = excl;
       int s = lo;
       for (; s < hi; ++s) {
-        if (cum + seg_w[s] > target) break;
-        cum += seg_w[s];
+        if (cum + static_cast<double>(seg_w[s]) > target) break;
+        cum += static_cast<double>(seg_w[s]);
       }
       seg = (s < hi) ? s : hi - 1;
-      cb = (s < hi) ? cum : cum - seg_w[hi - 1];
+      cb = (s < hi) ? cum : cum - static_cast<double>(seg_w[hi - 1]);
     }
     seg = __shfl_sync(0xffffffffu, seg, L);
     cb = __shfl_sync(0xffffffffu, cb, L);
     found = true;
   } else {
     int last = -1;
-    for (int s = lo; s < hi; ++s) if (seg_w[s] > 0.0) last = s;
+    for (int s = lo; s < hi; ++s) if (seg_w[s] > 0.f) last = s;
     const unsigned mm = __ballot_sync(0xffffffffu, last >= 0);
     const int L = mm ? 31 - __clz(mm) : 0;
     seg = __shfl_sync(0xffffffffu, last, L);
@@ -247,15 +248,12 @@ __device__ void slice_search(const float* zr, const float* qr, bool zvec, bool q
   const int e0 = (seg0 + seg) * kSeg + lane * 4;
   const float4 zv = load4(zr, e0, V, zvec, -INFINITY);
   float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (resid) qv = load4(qr, e0, V, qvec, 0.f);
-  const float wm = sh.seg_m[seg];
-  const float fs = static_cast<float>(resid ? sh.seg_f[seg] * inv_s : sh.seg_f[seg]);
-  const float cf = static_cast<float>(cpar);
+  if (f.resid) qv = load4(qr, e0, V, qvec, 0.f);
   double w[4];
-  w[0] = (e0 + 0 < V) ? static_cast<double>(elem_weight(zv.x, qv.x, wm, fs, invtau, cf, resid)) : 0.0;
-  w[1] = (e0 + 1 < V) ? static_cast<double>(elem_weight(zv.y, qv.y, wm, fs, invtau, cf, resid)) : 0.0;
-  w[2] = (e0 + 2 < V) ? static_cast<double>(elem_weight(zv.z, qv.z, wm, fs, invtau, cf, resid)) : 0.0;
-  w[3] = (e0 + 3 < V) ? static_cast<double>(elem_weight(zv.w, qv.w, wm, fs, invtau, cf, resid)) : 0.0;
+  w[0] = weight(zv.x, qv.x, f.k, f.zoff, f.inv_s, f.c, f.resid);
+  w[1] = weight(zv.y, qv.y, f.k, f.zoff, f.inv_s, f.c, f.resid);
+  w[2] = weight(zv.z, qv.z, f.k, f.zoff, f.inv_s, f.c, f.resid);
+  w[3] = weight(zv.w, qv.w, f.k, f.zoff, f.inv_s, f.c, f.resid);
   int t = -1;
   double margin = 0.0;
   if (found) {
@@ -283,7 +281,7 @@ __device__ void slice_search(const float* zr, const float* qr, bool zvec, bool q
   }
   if (t < 0) {
     int lp = -1;
-    for (int k = 0; k < 4; ++k) if (w[k] > 0.0) lp = e0 + k;
+    for (int k = 0; k < 4; ++k) if (w[k] > 0.0 && e0 + k < V) lp = e0 + k;
     const unsigned mm = __ballot_sync(0xffffffffu, lp >= 0);
     const int L = mm ? 31 - __clz(mm) : 0;
     t = __shfl_sync(0xffffffffu, lp, L);
@@ -388,22 +386,37 @@ accept_node_kernel(AcceptParams p) {
   Slot all[8];
   AcceptDec d;
   d.child = -1; d.token = -1; d.margin = INFINITY;
+  const bool greedy = (p.mode == TV_ACCEPT_GREEDY);
+  const bool specsample = (p.mode == TV_ACCEPT_SPECSAMPLE);
+  int has_child = 0;
+  if (specsample) {
+    int fl = 0;
+    for (int j = c + 1 + tid; j < n && !fl; j += blockDim.x) fl = (par[j] == c);
+    has_child = __syncthreads_or(fl);
+  }
+  const bool read_q = specsample && has_child;
+  const float* qr = read_q ? p.q + b * p.q_sb + c * p.q_st : nullptr;
+  const bool qvec = read_q && ((reinterpret_cast<uintptr_t>(qr) & 15u) == 0);
 
-  if (p.mode == TV_ACCEPT_GREEDY) {
-    float bv = -INFINITY;
-    int bi = INT_MAX;
-    bool nan = false;
-    for (int base = warp; base < nloc; base += kAcceptWarps * kUnroll) {
-      float4 v[kUnroll];
+  // ---- pass A: the row maximum (greedy: its first index), finiteness
+  float bv = -INFINITY;
+  int bi = INT_MAX;
+  bool bad = false;
+  for (int base = warp; base < nloc; base += kAcceptWarps * kUnroll) {
+    float4 v[kUnroll], qv[kUnroll];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int s = base + u * kAcceptWarps;
-        if (s < nloc) v[u] = load4(zr, (seg0 + s) * kSeg + lane * 4, V, zvec, -INFINITY);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int s = base + u * kAcceptWarps;
+      if (s < nloc) {
+        const int e0 = (seg0 + s) * kSeg + lane * 4;
+        v[u] = load4(zr, e0, V, zvec, -INFINITY);
+        if (read_q) qv[u] = load4(qr, e0, V, qvec, 0.f);
       }
+    }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int s = base + u * kAcceptWarps;
-        if (s >= nloc) break;
+    for (int u = 0; u < kUnroll; ++u) {
+      const int s = base + u * kAcceptWarps;
+      if (s < nloc) {
         const int e0 = (seg0 + s) * kSeg + lane * 4;
         const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
@@ -411,242 +424,176 @@ accept_node_kernel(AcceptParams p) {
           const int idx = e0 + k;
           if (idx < V) {
             const float x = xs[k];
-            if (isnan(x)) nan = true;
+            if (greedy ? isnan(x) : !isfinite(x)) bad = true;
             else if (x > bv || (x == bv && idx < bi)) { bv = x; bi = idx; }
           }
         }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-    }
-    const int any_nan = __syncthreads_or(nan ? 1 : 0);
-    if (lane == 0) { sh.red_f[warp] = bv; sh.red_i[warp] = bi; }
-    __syncthreads();
-    Slot mine;
-    mine.a = 0.0; mine.b = 0.0; mine.f = -INFINITY; mine.i = INT_MAX; mine.j = any_nan;
-    if (tid == 0) {
-      float v = -INFINITY;
-      int i = INT_MAX;
-      for (int w = 0; w < kAcceptWarps; ++w)
-        if (sh.red_f[w] > v || (sh.red_f[w] == v && sh.red_i[w] < i)) { v = sh.red_f[w]; i = sh.red_i[w]; }
-      mine.f = v; mine.i = i;
-    }
-    cluster_gather(cl, sh, mine, C, kred, all);
-    float gv = -INFINITY;
-    int a = INT_MAX, gnan = 0;
-    for (int r = 0; r < C; ++r) {
-      gnan |= all[r].j;
-      if (all[r].f > gv || (all[r].f == gv && all[r].i < a)) { gv = all[r].f; a = all[r].i; }
-    }
-    if (gnan) {
-      d.token = kNonFiniteRow;
-    } else if (rank == 0) {
-      d.child = first_child_with_token(par, tok, c, n, a, sh);
-      d.token = (d.child >= 0) ? -1 : a;
-    }
-  } else {
-    const bool specsample = (p.mode == TV_ACCEPT_SPECSAMPLE);
-    int has_child = 0;
-    if (specsample) {
-      int f = 0;
-      for (int j = c + 1 + tid; j < n && !f; j += blockDim.x) f = (par[j] == c);
-      has_child = __syncthreads_or(f);
-    }
-    const bool read_q = specsample && has_child;
-    const float* qr = read_q ? p.q + b * p.q_sb + c * p.q_st : nullptr;
-    const bool qvec = read_q && ((reinterpret_cast<uintptr_t>(qr) & 15u) == 0);
-    double* seg_w = sh.seg_w;
-    double* seg_r = sh.seg_r;
-    const double invtau = 1.0 / static_cast<double>(p.tau);
-    const float invtau_f = 1.0f / p.tau;
-
-    // pass 1: segment maxima and segment-frame exponential sums
-    bool bad = false, qbad = false;
-    float lmax = -INFINITY;
-    for (int base = warp; base < nloc; base += kAcceptWarps * kUnroll) {
-      float4 v[kUnroll], qv[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int s = base + u * kAcceptWarps;
-        if (s < nloc) {
-          const int e0 = (seg0 + s) * kSeg + lane * 4;
-          v[u] = load4(zr, e0, V, zvec, -INFINITY);
-          if (read_q) qv[u] = load4(qr, e0, V, qvec, 0.f);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int s = base + u * kAcceptWarps;
-        if (s >= nloc) break;
-        const int e0 = (seg0 + s) * kSeg + lane * 4;
-        const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-        float m4 = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (e0 + k < V) {
-            if (!isfinite(xs[k])) bad = true;
-            else m4 = fmaxf(m4, xs[k]);
-          }
         if (read_q) {
           const float qs[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            if (e0 + k < V && !(qs[k] >= 0.f && isfinite(qs[k]))) qbad = true;
+            if (e0 + k < V && !(qs[k] >= 0.f && isfinite(qs[k]))) bad = true;
         }
-        const float wm = warp_max(m4);
-        float af = 0.f;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (e0 + k < V && isfinite(xs[k])) af += expf((xs[k] - wm) * invtau_f);
-        const double a = warp_sum(static_cast<double>(af));
-        if (lane == 0) { sh.seg_m[s] = wm; seg_w[s] = a; }
-        lmax = fmaxf(lmax, wm);
       }
     }
-    const int any_bad = __syncthreads_or((bad || qbad) ? 1 : 0);
-    lmax = warp_max(lmax);
-    if (lane == 0) sh.red_f[warp] = lmax;
-    __syncthreads();
-    float cmax = -INFINITY;
-    for (int w = 0; w < kAcceptWarps; ++w) cmax = fmaxf(cmax, sh.red_f[w]);
-    // this CTA's sum in the frame of its own maximum
-    double part = 0.0;
-    for (int s = tid; s < nloc; s += blockDim.x)
-      part += seg_w[s] * exp((static_cast<double>(sh.seg_m[s]) - static_cast<double>(cmax)) * invtau);
-    const double csum = block_sum_d(part, sh);
-    Slot mine;
-    mine.a = csum; mine.b = 0.0; mine.f = cmax; mine.i = 0; mine.j = any_bad;
-    cluster_gather(cl, sh, mine, C, kred, all);
-    float M = -INFINITY;
-    int gbad = 0;
-    for (int r = 0; r < C; ++r) { M = fmaxf(M, all[r].f); gbad |= all[r].j; }
-    if (gbad) {
-      d.token = kNonFiniteRow;
-    } else {
-      double ssum = 0.0;
-      for (int r = 0; r < C; ++r)
-        if (all[r].f > -INFINITY)
-          ssum += all[r].a * exp((static_cast<double>(all[r].f) - static_cast<double>(M)) * invtau);
-      for (int s = tid; s < nloc; s += blockDim.x) {
-        const double f = exp((static_cast<double>(sh.seg_m[s]) - static_cast<double>(M)) * invtau);
-        sh.seg_f[s] = f;
-        seg_w[s] *= f;
-      }
-      // slice totals of the unnormalised softmax in the row frame
-      for (int r = 0; r < C; ++r)
-        sh.rank_tot[r] = (all[r].f > -INFINITY)
-                             ? all[r].a * exp((static_cast<double>(all[r].f) - static_cast<double>(M)) * invtau)
-                             : 0.0;
-      __syncthreads();
-      const double inv_s = 1.0 / ssum;
-      double margin = INFINITY;
-      bool decided = false;
-      double cpar = 0.0, D = 1.0;
-      bool resid = false;
-      if (specsample && has_child) {
-        const float* q = qr;
-        int k = 0;   // child ordinal = draw index
-        for (int base = c + 1; base < n && !decided; base += blockDim.x) {
-          const int j = base + tid;
-          const bool is = (j < n) && par[j] == c;
-          const unsigned m = __ballot_sync(0xffffffffu, is);
-          if (lane == 0) sh.red_i[warp] = __popc(m);
-          __syncthreads();
-          if (warp == 0) {
-            const int v = (lane < kAcceptWarps) ? sh.red_i[lane] : 0;
-            int incl = v;
+  }
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const int t = __shfl_up_sync(0xffffffffu, incl, o);
-              if (lane >= o) incl += t;
-            }
-            if (lane < kAcceptWarps) sh.wofs[lane] = incl - v;
-            if (lane == 31) sh.bc_int[3] = incl;
-          }
-          __syncthreads();
-          if (is) sh.clist[sh.wofs[warp] + __popc(m & ((1u << lane) - 1u))] = j;
-          const int cnt = sh.bc_int[3];
-          __syncthreads();
-          for (int ci = 0; ci < cnt && !decided; ++ci, ++k) {
-            const int jc = sh.clist[ci];
-            const int x = tok[jc];
-            if (x < 0 || x >= V) continue;
-            // point value of the current distribution at x, in the row frame
-            const double px = exp((static_cast<double>(zr[x]) - static_cast<double>(M)) * invtau) * inv_s;
-            const double qx = static_cast<double>(q[x]);
-            const double num = px - cpar * qx;
-            const double rx = num > 0.0 ? num / D : 0.0;
-            const double ratio = qx > 0.0 ? rx / qx : (rx > 0.0 ? INFINITY : 0.0);
-            const double u = accept_uniform(p.seed, p.step, b, c, k, kTagChild);
-            if (isfinite(ratio)) margin = fmin(margin, fabs(u - ratio));
-            if (u < ratio) {
-              d.child = jc;
-              decided = true;
-              break;
-            }
-            const double cn = cpar + D;
-            const double S_loc = residual_pass(zr, q, zvec, qvec, V, seg0, nloc, sh, seg_r, invtau_f, inv_s, cn, sh);
-            Slot ms;
-            ms.a = S_loc; ms.b = 0.0; ms.f = 0.f; ms.i = 0; ms.j = 0;
-            cluster_gather(cl, sh, ms, C, kred, all);
-            double S = 0.0;
-            for (int r = 0; r < C; ++r) S += all[r].a;
-            if (S > 0.0) {
-              cpar = cn; D = S; resid = true;
-              double* t = seg_w; seg_w = seg_r; seg_r = t;
-              for (int r = 0; r < C; ++r) sh.rank_tot[r] = all[r].a;
-            }
-            __syncthreads();
-          }
-        }
-      }
-      if (!decided) {
-        // inverse-CDF sample over the current weights: find the CTA whose
-        // slice holds the crossing, search inside it, gather the result
-        const int tag = specsample ? kTagResidual : kTagSpecExec;
-        const double u = accept_uniform(p.seed, p.step, b, c, 0, tag);
-        double W = 0.0;
-        for (int r = 0; r < C; ++r) W += sh.rank_tot[r];
-        const double target = u * W;
-        int owner = -1, last_pos = -1;
-        double base = 0.0, cum = 0.0;
-        for (int r = 0; r < C; ++r) {
-          if (sh.rank_tot[r] > 0.0) last_pos = r;
-          if (owner < 0 && cum + sh.rank_tot[r] > target) { owner = r; base = cum; }
-          if (owner < 0) cum += sh.rank_tot[r];
-        }
-        if (owner < 0) {                       // rounding: the last slice with weight
-          owner = last_pos < 0 ? 0 : last_pos;
-          base = 0.0;
-          for (int r = 0; r < owner; ++r) base += sh.rank_tot[r];
-        }
-        Slot res;
-        res.a = 0.0; res.b = 0.0; res.f = 0.f; res.i = -1; res.j = 0;
-        if (rank == owner && warp == 0) {
-          int t;
-          double mg;
-          slice_search(zr, qr, zvec, qvec, V, seg0, nloc, sh, seg_w, invtau_f, inv_s, cpar, resid, base,
-                       target, W, &t, &mg);
-          if (lane == 0) { sh.bc_int[2] = t; sh.bc_dbl[2] = mg; }
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+  }
+  const int any_bad = __syncthreads_or(bad ? 1 : 0);
+  if (lane == 0) { sh.red_f[warp] = bv; sh.red_i[warp] = bi; }
+  __syncthreads();
+  {
+    float v = -INFINITY;
+    int i = INT_MAX;
+#pragma unroll
+    for (int w = 0; w < kAcceptWarps; ++w)
+      if (sh.red_f[w] > v || (sh.red_f[w] == v && sh.red_i[w] < i)) { v = sh.red_f[w]; i = sh.red_i[w]; }
+    Slot mine;
+    mine.a = 0.0; mine.b = 0.0; mine.f = v; mine.i = i; mine.j = any_bad;
+    cluster_gather(cl, sh, mine, C, kred, all);
+  }
+  float M = -INFINITY;
+  int am = INT_MAX, gbad = 0;
+  for (int r = 0; r < C; ++r) {
+    gbad |= all[r].j;
+    if (all[r].f > M || (all[r].f == M && all[r].i < am)) { M = all[r].f; am = all[r].i; }
+  }
+
+  if (gbad) {
+    d.token = kNonFiniteRow;
+  } else if (greedy) {
+    if (rank == 0) {
+      d.child = first_child_with_token(par, tok, c, n, am, sh);
+      d.token = (d.child >= 0) ? -1 : am;
+    }
+  } else {
+    // ---- pass B: unnormalised softmax weights e_t in the row frame
+    const double k_d = 1.4426950408889634 / static_cast<double>(p.tau);
+    Frame f;
+    f.k = static_cast<float>(k_d);
+    f.zoff = -M * f.k;
+    f.inv_s = 1.f;
+    f.c = 0.f;
+    f.resid = false;
+    float* seg_w = sh.seg_a;
+    float* seg_r = sh.seg_b;
+    const double tot = weight_pass<false>(zr, nullptr, zvec, false, V, seg0, nloc, f, seg_w, sh);
+    {
+      Slot mine;
+      mine.a = tot; mine.b = 0.0; mine.f = 0.f; mine.i = 0; mine.j = 0;
+      cluster_gather(cl, sh, mine, C, kred, all);
+    }
+    double ssum = 0.0;
+    for (int r = 0; r < C; ++r) { ssum += all[r].a; sh.rank_tot[r] = all[r].a; }
+    __syncthreads();
+    const double inv_s = 1.0 / ssum;
+    // the weights e_t carry the fp32 frame offset zoff; point values use the
+    // same offset in fp64: p(x) = 2^(z_x k + zoff) / s
+    const double zoff_d = static_cast<double>(f.zoff);
+    const double k_f = static_cast<double>(f.k);
+    double margin = INFINITY;
+    bool decided = false;
+    double cpar = 0.0, D = 1.0;
+    if (read_q) {
+      const float* q = qr;
+      int kk = 0;   // child ordinal = draw index
+      for (int base = c + 1; base < n && !decided; base += blockDim.x) {
+        const int j = base + tid;
+        const bool is = (j < n) && par[j] == c;
+        const unsigned m = __ballot_sync(0xffffffffu, is);
+        if (lane == 0) sh.red_i[warp] = __popc(m);
+        __syncthreads();
+        if (tid == 0) {
+          int acc = 0;
+          for (int w = 0; w < kAcceptWarps; ++w) { sh.wofs[w] = acc; acc += sh.red_i[w]; }
+          sh.bc_int[3] = acc;
         }
         __syncthreads();
-        if (rank == owner) { res.i = sh.bc_int[2]; res.b = sh.bc_dbl[2]; }
-        cluster_gather(cl, sh, res, C, kred, all);
-        const int t = all[owner].i;
-        margin = fmin(margin, all[owner].b);
-        if (specsample) {
-          d.token = t;
-        } else if (rank == 0) {
-          d.child = first_child_with_token(par, tok, c, n, t, sh);
-          d.token = (d.child >= 0) ? -1 : t;
+        if (is) sh.clist[sh.wofs[warp] + __popc(m & ((1u << lane) - 1u))] = j;
+        const int cnt = sh.bc_int[3];
+        __syncthreads();
+        for (int ci = 0; ci < cnt && !decided; ++ci, ++kk) {
+          const int jc = sh.clist[ci];
+          const int x = tok[jc];
+          if (x < 0 || x >= V) continue;
+          const double px = exp2(static_cast<double>(zr[x]) * k_f + zoff_d) * inv_s;
+          const double qx = static_cast<double>(q[x]);
+          const double num = px - cpar * qx;
+          const double rx = num > 0.0 ? num / D : 0.0;
+          const double ratio = qx > 0.0 ? rx / qx : (rx > 0.0 ? INFINITY : 0.0);
+          const double u = accept_uniform(p.seed, p.step, b, c, kk, kTagChild);
+          if (isfinite(ratio)) margin = fmin(margin, fabs(u - ratio));
+          if (u < ratio) {
+            d.child = jc;
+            decided = true;
+            break;
+          }
+          // residual pass with c' = c + D
+          const double cn = cpar + D;
+          Frame fr = f;
+          fr.inv_s = static_cast<float>(inv_s);
+          fr.c = static_cast<float>(cn);
+          fr.resid = true;
+          const double S_loc = weight_pass<true>(zr, q, zvec, qvec, V, seg0, nloc, fr, seg_r, sh);
+          Slot ms;
+          ms.a = S_loc; ms.b = 0.0; ms.f = 0.f; ms.i = 0; ms.j = 0;
+          cluster_gather(cl, sh, ms, C, kred, all);
+          double S = 0.0;
+          for (int r = 0; r < C; ++r) S += all[r].a;
+          if (S > 0.0) {
+            cpar = cn; D = S; f = fr;
+            float* t = seg_w; seg_w = seg_r; seg_r = t;
+            for (int r = 0; r < C; ++r) sh.rank_tot[r] = all[r].a;
+          }
+          __syncthreads();
         }
       }
-      d.margin = margin;
     }
+    if (!decided) {
+      // inverse-CDF sample over the current weights: find the CTA whose
+      // slice holds the crossing, search inside it, gather the result
+      const int tag = specsample ? kTagResidual : kTagSpecExec;
+      const double u = accept_uniform(p.seed, p.step, b, c, 0, tag);
+      double W = 0.0;
+      for (int r = 0; r < C; ++r) W += sh.rank_tot[r];
+      const double target = u * W;
+      int owner = -1, last_pos = -1;
+      double base = 0.0, cum = 0.0;
+      for (int r = 0; r < C; ++r) {
+        if (sh.rank_tot[r] > 0.0) last_pos = r;
+        if (owner < 0 && cum + sh.rank_tot[r] > target) { owner = r; base = cum; }
+        if (owner < 0) cum += sh.rank_tot[r];
+      }
+      if (owner < 0) {                         // rounding: the last slice with weight
+        owner = last_pos < 0 ? 0 : last_pos;
+        base = 0.0;
+        for (int r = 0; r < owner; ++r) base += sh.rank_tot[r];
+      }
+      if (rank == owner && warp == 0) {
+        int t;
+        double mg;
+        slice_search(zr, qr, zvec, qvec, V, seg0, nloc, seg_w, f, base, target, W, &t, &mg);
+        if (lane == 0) { sh.bc_int[2] = t; sh.bc_dbl[2] = mg; }
+      }
+      __syncthreads();
+      Slot res;
+      res.a = 0.0; res.b = 0.0; res.f = 0.f; res.i = -1; res.j = 0;
+      if (rank == owner) { res.i = sh.bc_int[2]; res.b = sh.bc_dbl[2]; }
+      cluster_gather(cl, sh, res, C, kred, all);
+      const int t = all[owner].i;
+      margin = fmin(margin, all[owner].b);
+      if (specsample) {
+        d.token = t;
+      } else if (rank == 0) {
+        d.child = first_child_with_token(par, tok, c, n, t, sh);
+        d.token = (d.child >= 0) ? -1 : t;
+      }
+    }
+    d.margin = margin;
   }
   // rank 0 publishes the decision; the last node of the sequence walks
   if (rank == 0) {
