@@ -70,7 +70,7 @@ struct AcceptParams {
 constexpr int kAcceptThreads = 256;
 constexpr int kAcceptWarps = kAcceptThreads / kWarp;
 constexpr int kSeg = 128;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 2;
 constexpr int kMaxSegPerCta = 512;      // 65536 elements per CTA
 
 // ------------------------------------------------------------ shared state
