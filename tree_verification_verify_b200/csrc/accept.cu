@@ -70,7 +70,7 @@ struct AcceptParams {
 constexpr int kAcceptThreads = 256;
 constexpr int kAcceptWarps = kAcceptThreads / kWarp;
 constexpr int kSeg = 128;
-constexpr int kUnroll = 2;
+constexpr int kUnroll = 4;
 constexpr int kMaxSegPerCta = 512;      // 65536 elements per CTA
 
 // ------------------------------------------------------------ shared state
@@ -336,17 +336,11 @@ __device__ void accept_walk(const AcceptParams& p, int b, int n, AcceptShared& s
   const int len = sh.bc_int[1];
   for (int i = len + threadIdx.x; i < T; i += blockDim.x) acc[i] = -1;
   for (int i = len + (walk ? 1 : 0) + threadIdx.x; i < T + 1; i += blockDim.x) out[i] = -1;
-  // leave the workspace zero: the next call may lay it out differently
-  if (walk) {
-    AcceptDec z;
-    z.child = 0; z.token = 0; z.margin = 0.0;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) p.dec[static_cast<int64_t>(b) * T + i] = z;
-  }
 }
 
 // ------------------------------------------------------------ node kernel
 
-__global__ void __launch_bounds__(kAcceptThreads, 4)
+__global__ void __launch_bounds__(kAcceptThreads, 3)
 accept_node_kernel(AcceptParams p) {
   __shared__ AcceptShared sh;
   cg::cluster_group cl = cg::this_cluster();
@@ -615,9 +609,12 @@ accept_node_kernel(AcceptParams p) {
 
 // ------------------------------------------------------------ host side
 
+// Workspace: [0, 64 KB) ticket counters (zero between calls), then the
+// per-node decisions.
+constexpr size_t kAcceptTicketBytes = 64 * 1024;
+
 size_t accept_workspace_bytes(int B, int T) {
-  const size_t dec = static_cast<size_t>(B) * static_cast<size_t>(T) * sizeof(AcceptDec);
-  return ((dec + 255) & ~static_cast<size_t>(255)) + static_cast<size_t>(B) * sizeof(int32_t);
+  return kAcceptTicketBytes + static_cast<size_t>(B) * static_cast<size_t>(T) * sizeof(AcceptDec);
 }
 
 cudaError_t launch_accept(const tv_accept_args* a, int mode, void* ws, cudaStream_t stream) {
@@ -632,9 +629,8 @@ cudaError_t launch_accept(const tv_accept_args* a, int mode, void* ws, cudaStrea
   p.tau = a->temperature;
   p.seed = a->seed; p.step = a->step;
   p.status = a->dev_status;
-  const size_t dec = static_cast<size_t>(a->B) * static_cast<size_t>(a->T) * sizeof(AcceptDec);
-  p.dec = static_cast<AcceptDec*>(ws);
-  p.ticket = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(ws) + ((dec + 255) & ~static_cast<size_t>(255)));
+  p.ticket = static_cast<int32_t*>(ws);
+  p.dec = reinterpret_cast<AcceptDec*>(static_cast<unsigned char*>(ws) + kAcceptTicketBytes);
   p.n_acc = a->n_accepted; p.acc_nodes = a->accepted_nodes; p.out_tokens = a->out_tokens;
   p.min_margin = a->min_margin;
   if (a->B == 0) return cudaSuccess;

@@ -31,7 +31,13 @@ struct AttnParams {
   float* part_o;               // [nchunk+1][B][T][Hq][d]
   float* part_lse;             // [nchunk+1][B][T][Hq]
   int32_t* node_ok;            // [B][T]
+  int32_t* tickets;            // per-group counters, zero between calls
 };
+
+// The first kTicketBytes of every workspace hold ticket counters that each
+// call returns to zero (so calls of any shape may share one workspace).
+constexpr size_t kTicketBytes = 64 * 1024;
+constexpr int kMaxTickets = static_cast<int>(kTicketBytes / sizeof(int32_t));
 
 __host__ __device__ inline int64_t part_row(const AttnParams& p, int chunk, int b, int i, int h) {
   return ((static_cast<int64_t>(chunk) * p.B + b) * p.T + i) * p.Hq + h;

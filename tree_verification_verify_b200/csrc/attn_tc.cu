@@ -1,21 +1,29 @@
-// tree_verify_attn, tensor-core prefix kernel for sm_100a (tcgen05 + TMEM +
-// TMA), bf16 with d = 128.
+// tree_verify_attn, tensor-core kernel for sm_100a (tcgen05 + TMEM + TMA),
+// bf16 with d = 128.
 //
-// Every draft node attends to the whole shared prefix (tree attention;
-// SpecExec page, "Approach": the whole tree is verified in one target pass),
-// so the prefix part is a dense contraction: the G query heads of one kv
-// head are packed with the tree nodes into M = 128 query rows (row r = node
-// r / G, head r % G; the "inter-draft-token reuse" of the sparse verification
-// page, "Methodology" 4: every K/V tile is loaded once for all nodes and
-// heads of the tile).  One CTA owns (sequence, kv head, 128-row tile, prefix
-// chunk) and produces a partial (O, lse) that the log-sum-exp merge combines
-// with the other chunks and with the tree-ancestor partial.
+// Tree attention (SpecExec page, "Approach": the whole tree is verified in
+// one target pass): node i attends to the shared prefix and to its root
+// path.  The G query heads of one kv head are packed with the tree nodes
+// into M = 128 query rows (row r = node r / G, head r % G); every K/V tile
+// is loaded once for all nodes and heads of the tile (the "inter-draft-token
+// reuse" of the sparse verification page, "Methodology" 4).
+//
+// One CTA owns (sequence, kv head, 128-row tile, prefix chunk).  Its key
+// tiles are the chunk's prefix tiles of 128 keys and, in chunk 0, the tree
+// tiles: the union U of the tile's nodes' root paths, gathered into K/V
+// tiles and masked per row by an ancestor bitmask built in shared memory
+// from parent[] (slot of node a in U = number of marked nodes below a in a
+// node bitmap).  All tiles share one online softmax.  With a single chunk
+// the CTA writes the final output; otherwise every chunk writes a partial
+// (O, lse) and the last CTA of the group (an atomic ticket, no waiting)
+// merges them.
 //
 // Warp roles (192 threads):
 //   warps 0-3  softmax / correction / epilogue: thread t owns query row t,
 //              which is TMEM lane t (tcgen05.ld 32x32b);
-//   warp 4     TMA producer: Q once, then K and V tiles of 128 keys into a
-//              two-stage ring (128B-swizzled, K-major for K, MN-major for V);
+//   warp 4     producer: Q once, prefix K/V tiles by TMA into a two-stage
+//              ring (128B-swizzled; K-major for K, MN-major for V), the
+//              tree bookkeeping, and the gathered tree tiles (cp.async);
 //   warp 5     TMEM allocator and MMA issuer (one thread): S = Q K^T into one
 //              of two TMEM S buffers, O += P V into the TMEM O accumulator.
 // Online softmax in base 2 with a lazily updated row maximum: O and the row
@@ -39,12 +47,14 @@ constexpr int kRows = 128;          // M
 constexpr int kKeys = 128;          // keys per tile (N of QK, K of PV)
 constexpr int kD = 128;
 constexpr int kStages = 2;
+constexpr int kMaxT = 4096;         // tree nodes handled by this kernel
 constexpr uint32_t kHalfBytes = kRows * 128;            // 128 rows x 128 B
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;         // 32 KB (d = 128 bf16)
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemKV = kSmemQ + kTileBytes;       // stage s: K at +s*64K, V at +32K
 constexpr uint32_t kSmemP = kSmemKV + kStages * 2 * kTileBytes;
-constexpr uint32_t kSmemBytes = kSmemP + kTileBytes;    // 192 KB
+constexpr uint32_t kSmemU = kSmemP + kTileBytes;        // U list (int32, kMaxT)
+constexpr uint32_t kSmemBytes = kSmemU + kMaxT * 4;     // 208 KB
 constexpr uint32_t kTmemCols = 512;                     // S0, S1, O (128 each)
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr uint32_t kWaitLimit = 1u << 22;
@@ -57,9 +67,16 @@ struct Bars {
   uint64_t s_free[2];
   uint64_t p_full;
   uint64_t pv_done;
+  uint64_t tree_info;
   uint32_t tmem_base;
   int abort;
+  int nU;                           // nodes in the union of root paths
+  int last;                         // this CTA merges the group
+  uint32_t bm[kMaxT / 32];          // node bitmap of U
+  int pre[kMaxT / 32];              // marked nodes below each bitmap word
+  int node_ok[kRows];               // root path of the tile's node is well formed
 };
+
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -179,18 +196,54 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
-struct TcMaps {
-  CUtensorMap q, k, v;
-};
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Slot of node a in U: the number of marked nodes below a.
+__device__ __forceinline__ int u_slot(const Bars& bars, int a) {
+  return bars.pre[a >> 5] + __popc(bars.bm[a >> 5] & ((1u << (a & 31)) - 1u));
+}
+
+// Ancestor bitmask of node i (whose root path is well formed) over tree
+// tile tt, i.e. the slots [128 tt, 128 tt + 128) of U.
+__device__ __forceinline__ void tree_mask(const int32_t* par, int i, int tt, const Bars& bars, uint32_t* mk) {
+  mk[0] = mk[1] = mk[2] = mk[3] = 0u;
+  int j = i;
+  for (int step = 0; step <= i; ++step) {
+    const int sl = u_slot(bars, j);
+    if ((sl >> 7) == tt) mk[(sl >> 5) & 3] |= 1u << (sl & 31);
+    if (j == 0) break;
+    j = par[j];
+  }
+}
+
+// Whether node i's root path reaches node 0 through parent[j] in [0, j).
+__device__ __forceinline__ bool path_ok(const int32_t* par, int i) {
+  if (par[0] != -1) return false;
+  int j = i;
+  for (int step = 0; step <= i && j != 0; ++step) {
+    const int pj = par[j];
+    if (pj < 0 || pj >= j) return false;
+    j = pj;
+  }
+  return true;
+}
 
 }  // namespace tc
 
 using namespace tc;
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                      const __grid_constant__ CUtensorMap tmap_v, AttnParams p) {
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+               const __grid_constant__ CUtensorMap tmap_v, AttnParams p) {
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ Bars bars;
   const int chunk = blockIdx.x;
@@ -199,33 +252,30 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.G;
   const int n = p.n_nodes ? p.n_nodes[b] : p.T;
-  if (n < 0 || n > p.T) return;
+  if (n < 0 || n > p.T) {
+    if (chunk == 0 && tile == 0 && g == 0 && tid == 0) set_status(p.status, TV_DEV_BAD_LEN);
+    return;
+  }
   const int i0 = tile * (kRows / G);
   if (i0 >= n) return;
-  int L = p.prefix_len[b];
-  if (L < 0 || L > p.Lmax) L = 0;
+  const int32_t* par = p.parent + b * p.par_sb;
+  const int Lraw = p.prefix_len[b];
+  const bool bad_len = (Lraw < 0 || Lraw > p.Lmax);
+  const int L = bad_len ? 0 : Lraw;
   const int k0 = chunk * p.chunk_len;
   const int k1 = min(k0 + p.chunk_len, L);
+  const int nprefix = (k1 > k0) ? (k1 - k0 + kKeys - 1) / kKeys : 0;
+  const int nodes_here = min(kRows / G, n - i0);
   // this thread's query row (softmax warps)
   const int row_node = i0 + tid / G;
   const int row_head = g * G + tid % G;
-  const bool row_valid = tid < kRows && row_node < n;
-  if (k1 <= k0) {
-    // no prefix keys in this chunk: an empty partial
-    if (row_valid) {
-      const int64_t pr = part_row(p, chunk, b, row_node, row_head);
-      float* po = p.part_o + pr * kD;
-      for (int c = 0; c < kD; ++c) po[c] = 0.f;
-      p.part_lse[pr] = -INFINITY;
-    }
-    return;
-  }
-  const int ntiles = (k1 - k0 + kKeys - 1) / kKeys;
+  const bool row_valid = tid < kRows && (tid / G) < nodes_here;
 
   // 1024-aligned dynamic shared memory (128B swizzle atoms are 1 KB)
   const uint32_t raw = smem_u32(dsmem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = dsmem_raw + (base - raw);
+  int* ulist = reinterpret_cast<int*>(gbase + kSmemU);
   volatile int* abort = &bars.abort;
 
   if (tid == 0) {
@@ -234,7 +284,10 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
     for (int s = 0; s < 2; ++s) { mbar_init(&bars.s_full[s], 1); mbar_init(&bars.s_free[s], 4); }
     mbar_init(&bars.p_full, 4);
     mbar_init(&bars.pv_done, 1);
+    mbar_init(&bars.tree_info, 1);
     bars.abort = 0;
+    bars.nU = 0;
+    bars.last = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -249,29 +302,122 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
   __syncthreads();
   fence_after();
   const uint32_t tmem = bars.tmem_base;
+  const bool has_tree = (chunk == 0);
 
   if (warp == 4) {
-    // ---------------------------------------------------------------- TMA producer
+    // ---------------------------------------------------------------- producer
+    const int first = min(nprefix, kStages);
     if (lane == 0) {
       const uint32_t sq = base + kSmemQ;
       mbar_expect_tx(&bars.q_full, kTileBytes);
       tma_load_4d(&tmap_q, sq, &bars.q_full, 0, g * G, i0, b);
       tma_load_4d(&tmap_q, sq + kHalfBytes, &bars.q_full, 64, g * G, i0, b);
-      int issued = 0;
-      for (int j = 0; j < ntiles; ++j) {
-        const int s = j % kStages;
-        if (j >= kStages && !mbar_wait(&bars.empty[s], ((j / kStages) - 1) & 1, abort)) break;
-        const uint32_t sk = base + kSmemKV + s * 2 * kTileBytes;
-        const uint32_t sv = sk + kTileBytes;
+      for (int j = 0; j < first; ++j) {
+        const uint32_t sk = base + kSmemKV + j * 2 * kTileBytes;
         const int kb = k0 + j * kKeys;
-        mbar_expect_tx(&bars.full[s], 2 * kTileBytes);
-        tma_load_4d(&tmap_k, sk, &bars.full[s], 0, g, kb, b);
-        tma_load_4d(&tmap_k, sk + kHalfBytes, &bars.full[s], 64, g, kb, b);
-        tma_load_4d(&tmap_v, sv, &bars.full[s], 0, g, kb, b);
-        tma_load_4d(&tmap_v, sv + kHalfBytes, &bars.full[s], 64, g, kb, b);
-        ++issued;
+        mbar_expect_tx(&bars.full[j], 2 * kTileBytes);
+        tma_load_4d(&tmap_k, sk, &bars.full[j], 0, g, kb, b);
+        tma_load_4d(&tmap_k, sk + kHalfBytes, &bars.full[j], 64, g, kb, b);
+        tma_load_4d(&tmap_v, sk + kTileBytes, &bars.full[j], 0, g, kb, b);
+        tma_load_4d(&tmap_v, sk + kTileBytes + kHalfBytes, &bars.full[j], 64, g, kb, b);
       }
-      // drain: every issued load must land before the CTA can exit
+    }
+    int ntree = 0;
+    if (has_tree) {
+      // union U of the root paths of this tile's nodes, as a node bitmap
+      const int nw = (n + 31) >> 5;
+      for (int w = lane; w < nw; w += 32) bars.bm[w] = 0u;
+      __syncwarp();
+      for (int r = lane; r < nodes_here; r += 32) {
+        const int i = i0 + r;
+        int ok = (par[0] == -1) ? 1 : 0;
+        int j = i;
+        for (int step = 0; step <= i; ++step) {
+          atomicOr(&bars.bm[j >> 5], 1u << (j & 31));
+          if (j == 0) break;
+          const int pj = par[j];
+          if (pj < 0 || pj >= j) { ok = 0; break; }
+          j = pj;
+        }
+        bars.node_ok[r] = ok;
+      }
+      __syncwarp();
+      // prefix counts per bitmap word, then the U list in node order
+      const int per = (nw + 31) / 32;
+      const int lo = min(lane * per, nw), hi = min(lo + per, nw);
+      int cnt = 0;
+      for (int w = lo; w < hi; ++w) cnt += __popc(bars.bm[w]);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int run = incl - cnt;
+      for (int w = lo; w < hi; ++w) {
+        bars.pre[w] = run;
+        uint32_t m = bars.bm[w];
+        while (m) {
+          const int bit = __ffs(m) - 1;
+          ulist[run++] = w * 32 + bit;
+          m &= m - 1u;
+        }
+      }
+      if (lane == 31) bars.nU = incl;
+      __syncwarp();
+      ntree = (bars.nU + kKeys - 1) / kKeys;
+      if (lane == 0) mbar_arrive(&bars.tree_info);
+    }
+    const int ntot = nprefix + ntree;
+    int issued = first;
+    for (int j = first; j < ntot; ++j) {
+      const int s = j % kStages;
+      bool ok = true;
+      if (j >= kStages) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&bars.empty[s], ((j / kStages) - 1) & 1, abort);
+        ok = __all_sync(0xffffffffu, w);
+      }
+      if (!ok) break;
+      const uint32_t sk = base + kSmemKV + s * 2 * kTileBytes;
+      if (j < nprefix) {
+        if (lane == 0) {
+          const int kb = k0 + j * kKeys;
+          mbar_expect_tx(&bars.full[s], 2 * kTileBytes);
+          tma_load_4d(&tmap_k, sk, &bars.full[s], 0, g, kb, b);
+          tma_load_4d(&tmap_k, sk + kHalfBytes, &bars.full[s], 64, g, kb, b);
+          tma_load_4d(&tmap_v, sk + kTileBytes, &bars.full[s], 0, g, kb, b);
+          tma_load_4d(&tmap_v, sk + kTileBytes + kHalfBytes, &bars.full[s], 64, g, kb, b);
+        }
+      } else {
+        // gathered tree tile: rows = U[128 tt ..], 128B-swizzled like TMA writes
+        const int tt = j - nprefix;
+        const int nU = bars.nU;
+        const __nv_bfloat16* kt = static_cast<const __nv_bfloat16*>(p.kt);
+        const __nv_bfloat16* vt = static_cast<const __nv_bfloat16*>(p.vt);
+        for (int e = lane; e < kRows * 16; e += 32) {
+          const int r = e >> 4, c = e & 15;
+          const int slot = tt * kKeys + r;
+          const uint32_t off = static_cast<uint32_t>(c >> 3) * kHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+          if (slot < nU) {
+            const int a = ulist[slot];
+            const int64_t src = b * p.kt_sb + static_cast<int64_t>(a) * p.kt_st + g * p.kt_sh + c * 8;
+            cp_async16(sk + off, kt + src);
+            cp_async16(sk + kTileBytes + off, vt + src);
+          } else {
+            *reinterpret_cast<uint4*>(gbase + (sk - base) + off) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(gbase + (sk - base) + kTileBytes + off) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        cp_async_wait_all();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.full[s]);
+      }
+      ++issued;
+    }
+    // drain: every issued load must land before the CTA can exit
+    if (lane == 0) {
       mbar_wait(&bars.q_full, 0, abort);
       for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
         uint32_t it = 0;
@@ -279,16 +425,22 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
         }
       }
     }
+    __syncwarp();
   } else if (warp == 5) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
+      bool ok = true;
+      int ntot = nprefix;
+      if (has_tree) {
+        ok = mbar_wait(&bars.tree_info, 0, abort);
+        ntot += (bars.nU + kKeys - 1) / kKeys;
+      }
       const uint32_t idesc_qk = instr_desc(kRows, kKeys, 0, 0);
       const uint32_t idesc_pv = instr_desc(kRows, kD, 0, 1);
       const uint32_t sq = base + kSmemQ, sp = base + kSmemP;
-      bool ok = mbar_wait(&bars.q_full, 0, abort);
-      // S(0)
-      if (ok) ok = mbar_wait(&bars.full[0], 0, abort);
-      if (ok) {
+      if (ok && ntot > 0) ok = mbar_wait(&bars.q_full, 0, abort);
+      if (ok && ntot > 0) ok = mbar_wait(&bars.full[0], 0, abort);
+      if (ok && ntot > 0) {
         fence_after();
         const uint32_t sk = base + kSmemKV;
 #pragma unroll
@@ -299,9 +451,8 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
         }
         mma_commit(&bars.s_full[0]);
       }
-      for (int j = 0; j < ntiles && ok; ++j) {
-        // S(j+1) into the other buffer while the softmax works on S(j)
-        if (j + 1 < ntiles) {
+      for (int j = 0; j < ntot && ok; ++j) {
+        if (j + 1 < ntot) {
           const int s1 = (j + 1) % kStages;
           ok = mbar_wait(&bars.full[s1], ((j + 1) / kStages) & 1, abort);
           if (ok && j >= 1) ok = mbar_wait(&bars.s_free[(j + 1) & 1], ((j - 1) >> 1) & 1, abort);
@@ -317,7 +468,6 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
           }
           mma_commit(&bars.s_full[(j + 1) & 1]);
         }
-        // O += P(j) V(j)
         ok = mbar_wait(&bars.p_full, j & 1, abort);
         if (!ok) break;
         fence_after();
@@ -339,9 +489,18 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      const int kb = k0 + j * kKeys;
-      const int nk = min(kKeys, k1 - kb);
+    int ntot = nprefix;
+    bool my_ok = true;
+    if (has_tree) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars.tree_info, 0, abort));
+      ntot += (bars.nU + kKeys - 1) / kKeys;
+      my_ok = row_valid && bars.node_ok[tid / G] != 0;
+    }
+    for (int j = 0; j < ntot && ok; ++j) {
+      const bool tree_tile = j >= nprefix;
+      const int nk = tree_tile ? 0 : min(kKeys, k1 - (k0 + j * kKeys));
+      uint32_t mk[4] = {0u, 0u, 0u, 0u};
+      if (tree_tile && my_ok) tree_mask(par, row_node, j - nprefix, bars, mk);
       ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full[j & 1], (j >> 1) & 1, abort));
       if (!ok) break;
       fence_after();
@@ -353,11 +512,11 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.s_free[j & 1]);
-      // row maximum over the valid keys of the tile
       float mt = -INFINITY;
 #pragma unroll
       for (int c = 0; c < kKeys; ++c) {
-        s[c] = (c < nk) ? s[c] * sl2 : -INFINITY;
+        const bool keep = tree_tile ? ((mk[c >> 5] >> (c & 31)) & 1u) != 0u : c < nk;
+        s[c] = keep ? s[c] * sl2 : -INFINITY;
         mt = fmaxf(mt, s[c]);
       }
       const float m_new = fmaxf(m_run, mt);
@@ -367,17 +526,17 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
       if (first) {
         m_run = m_new;
       } else if (grow) {
-        factor = exp2f(m_run - m_new);
+        factor = ex2_approx(m_run - m_new);
         m_run = m_new;
       }
+      const float mu = (m_run == -INFINITY) ? 0.f : m_run;
       float rs = 0.f;
 #pragma unroll
       for (int c = 0; c < kKeys; ++c) {
-        s[c] = exp2f(s[c] - m_run);
+        s[c] = ex2_approx(s[c] - mu);
         rs += s[c];
       }
       l_run = l_run * factor + rs;
-      // the previous PV must be done before O is rescaled and P rewritten
       if (j > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (j - 1) & 1, abort));
         if (!ok) break;
@@ -395,13 +554,13 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
           tmem_wait_st();
         }
       }
-      if (nk < kKeys) {
-        // ragged tile: V rows past the prefix end may hold anything; zero them
+      if (!tree_tile && nk < kKeys) {
+        // ragged prefix tile: V rows past the prefix end may hold anything
         ok = __all_sync(0xffffffffu, mbar_wait(&bars.full[j % kStages], (j / kStages) & 1, abort));
         if (!ok) break;
         if (tid >= nk) {
           uint8_t* sv = gbase + kSmemKV + (j % kStages) * 2 * kTileBytes + kTileBytes;
-          uint4 z = make_uint4(0u, 0u, 0u, 0u);
+          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             *reinterpret_cast<uint4*>(sv + tid * 128 + c * 16) = z;
@@ -409,7 +568,6 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
           }
         }
       }
-      // P row -> shared memory, bf16, 128B-swizzled K-major
       uint8_t* prow = gbase + kSmemP + tid * 128;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
@@ -426,27 +584,59 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.p_full);
     }
-    // epilogue: wait for the last PV, normalise, write the partial
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (ntiles - 1) & 1, abort));
+    // epilogue
+    if (ok && ntot > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (ntot - 1) & 1, abort));
     if (ok) {
       fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      float* po = row_valid ? p.part_o + part_row(p, chunk, b, row_node, row_head) * kD : nullptr;
+      const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+      if (p.nchunk == 1) {
+        // single chunk: this CTA holds the whole result
+        const bool good = my_ok && !bad_len;
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + row_node * p.o_st + row_head * p.o_sh;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float o[32];
-        tmem_ld32(trow + kColO + c * 32, o);
-        tmem_wait_ld();
-        if (row_valid) {
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(trow + kColO + c * 32, v);
+          tmem_wait_ld();
+          if (row_valid) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(po + c * 32 + e) =
-                make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
+            for (int e = 0; e < 32; e += 8) {
+              uint4 w;
+              if (good) {
+                w.x = pack_bf16(v[e] * inv, v[e + 1] * inv);
+                w.y = pack_bf16(v[e + 2] * inv, v[e + 3] * inv);
+                w.z = pack_bf16(v[e + 4] * inv, v[e + 5] * inv);
+                w.w = pack_bf16(v[e + 6] * inv, v[e + 7] * inv);
+              } else {
+                w.x = w.y = w.z = w.w = pack_bf16(NAN, NAN);
+              }
+              *reinterpret_cast<uint4*>(o + c * 32 + e) = w;
+            }
+          }
         }
+        if (row_valid) {
+          if (p.lse) p.lse[(static_cast<int64_t>(b) * p.T + row_node) * p.Hq + row_head] = good ? lse : NAN;
+          if (!my_ok) set_status(p.status, TV_DEV_BAD_PARENT);
+          if (bad_len && row_node == 0 && row_head == 0) set_status(p.status, TV_DEV_BAD_LEN);
+        }
+      } else {
+        float* po = row_valid ? p.part_o + part_row(p, chunk, b, row_node, row_head) * kD : nullptr;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(trow + kColO + c * 32, v);
+          tmem_wait_ld();
+          if (row_valid) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(po + c * 32 + e) =
+                  (l_run > 0.f) ? make_float4(v[e] * inv, v[e + 1] * inv, v[e + 2] * inv, v[e + 3] * inv)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        if (row_valid) p.part_lse[part_row(p, chunk, b, row_node, row_head)] = lse;
       }
-      if (row_valid)
-        p.part_lse[part_row(p, chunk, b, row_node, row_head)] =
-            l_run > 0.f ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
     }
   }
   // ------------------------------------------------------------------ teardown
@@ -454,13 +644,71 @@ attn_prefix_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_c
   __syncthreads();
   if (*abort) {
     if (tid == 0) set_status(p.status, TV_DEV_TIMEOUT);
-    if (row_valid) p.part_lse[part_row(p, chunk, b, row_node, row_head)] = NAN;
+    if (row_valid) {
+      if (p.nchunk == 1) {
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + row_node * p.o_st + row_head * p.o_sh;
+        for (int c = 0; c < kD; ++c) o[c] = __float2bfloat16(NAN);
+      } else {
+        p.part_lse[part_row(p, chunk, b, row_node, row_head)] = NAN;
+      }
+    }
   }
   if (warp == 5) {
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
+  if (p.nchunk == 1) return;
+  // ------------------------------------------------------------------ split merge
+  const int group = (b * p.Hkv + g) * gridDim.y + tile;
+  if (tid == 0) {
+    __threadfence();
+    const int done = atomicAdd(&p.tickets[group], 1);
+    bars.last = (done == p.nchunk - 1);
+  }
+  __syncthreads();
+  if (!bars.last || warp >= 4) return;
+  __threadfence();
+  // warp w merges rows 32w .. 32w+31; lane l first checks row 32w+l's path
+  const int myrow = warp * 32 + lane;
+  const bool mine_valid = (myrow / G) < nodes_here;
+  const bool mine_ok = mine_valid && path_ok(par, i0 + myrow / G);
+  const int np = p.nchunk;
+  for (int rr = 0; rr < 32; ++rr) {
+    const int r = warp * 32 + rr;
+    if (!__shfl_sync(0xffffffffu, mine_valid ? 1 : 0, rr)) continue;
+    const bool good = __shfl_sync(0xffffffffu, mine_ok ? 1 : 0, rr) && !bad_len;
+    const int node = i0 + r / G, head = g * G + r % G;
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + node * p.o_st + head * p.o_sh;
+    float lc = -INFINITY;
+    for (int c = lane; c < np; c += 32) lc = fmaxf(lc, __ldcg(&p.part_lse[part_row(p, c, b, node, head)]));
+    const float M = warp_max(lc);
+    const float wl = (lane < np && lc > -INFINITY) ? __expf(lc - M) : 0.f;
+    const float den = warp_sumf(wl);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < np; ++c) {
+      const float w = __shfl_sync(0xffffffffu, wl, c & 31);
+      if (w == 0.f) continue;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(p.part_o + part_row(p, c, b, node, head) * kD) + lane);
+      acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+    }
+    const float inv = 1.f / den;
+    uint2 wv;
+    if (good && den > 0.f) {
+      wv.x = pack_bf16(acc.x * inv, acc.y * inv);
+      wv.y = pack_bf16(acc.z * inv, acc.w * inv);
+    } else {
+      wv.x = wv.y = pack_bf16(NAN, NAN);
+    }
+    *reinterpret_cast<uint2*>(o + lane * 4) = wv;
+    if (lane == 0) {
+      if (p.lse) p.lse[(static_cast<int64_t>(b) * p.T + node) * p.Hq + head] = (good && den > 0.f) ? M + __logf(den) : NAN;
+      if (!good && !bad_len) set_status(p.status, TV_DEV_BAD_PARENT);
+      if (bad_len && node == 0 && head == 0) set_status(p.status, TV_DEV_BAD_LEN);
+    }
+  }
+  if (tid == 0) p.tickets[group] = 0;                // ready for the next call
 }
 
 // ------------------------------------------------------------------ host side
@@ -502,19 +750,22 @@ bool stride_ok(int64_t s) { return s > 0 && (s * 2) % 16 == 0 && s * 2 < (1ll <<
 bool attn_tc_supported(const tv_attn_args* a) {
   if (a->dtype != TV_BF16 || a->d != 128 || a->sparse_topk != 0) return false;
   if (a->B == 0 || a->T == 0 || a->Lmax == 0) return false;
+  if (a->T > kMaxT) return false;
   const int G = a->Hq / a->Hkv;
   if (G > 128 || 128 % G != 0) return false;
-  if (a->Lmax > (1 << 30) || a->T > (1 << 30)) return false;
+  if (a->Lmax > (1 << 30)) return false;
   if (!stride_ok(a->q_sh) || !stride_ok(a->q_st) || !stride_ok(a->q_sb)) return false;
   if (!stride_ok(a->kv_sh) || !stride_ok(a->kv_sl) || !stride_ok(a->kv_sb)) return false;
+  if (!stride_ok(a->kt_sh) || !stride_ok(a->kt_st) || !stride_ok(a->kt_sb)) return false;
+  if (!stride_ok(a->o_sh) || !stride_ok(a->o_st) || !stride_ok(a->o_sb)) return false;
   const uintptr_t al = reinterpret_cast<uintptr_t>(a->q) | reinterpret_cast<uintptr_t>(a->k_cache) |
-                       reinterpret_cast<uintptr_t>(a->v_cache);
+                       reinterpret_cast<uintptr_t>(a->v_cache) | reinterpret_cast<uintptr_t>(a->k_tree) |
+                       reinterpret_cast<uintptr_t>(a->v_tree) | reinterpret_cast<uintptr_t>(a->out);
   if (al & 15u) return false;
   if (!encode_fn()) return false;
   {
     CUtensorMap m;
-    const int G2 = a->Hq / a->Hkv;
-    if (!make_map(&m, a->q, a->d, a->Hq, a->T, a->B, a->q_sh, a->q_st, a->q_sb, G2, kRows / G2) ||
+    if (!make_map(&m, a->q, a->d, a->Hq, a->T, a->B, a->q_sh, a->q_st, a->q_sb, G, kRows / G) ||
         !make_map(&m, a->k_cache, a->d, a->Hkv, a->Lmax, a->B, a->kv_sh, a->kv_sl, a->kv_sb, 1, kKeys) ||
         !make_map(&m, a->v_cache, a->d, a->Hkv, a->Lmax, a->B, a->kv_sh, a->kv_sl, a->kv_sb, 1, kKeys))
       return false;
@@ -527,19 +778,19 @@ bool attn_tc_supported(const tv_attn_args* a) {
 }
 
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream) {
-  TcMaps maps;
+  CUtensorMap mq, mk, mv;
   const int G = p.G;
-  if (!make_map(&maps.q, p.q, p.d, p.Hq, p.T, p.B, p.q_sh, p.q_st, p.q_sb, G, kRows / G) ||
-      !make_map(&maps.k, p.kc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, kKeys) ||
-      !make_map(&maps.v, p.vc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, kKeys))
+  if (!make_map(&mq, p.q, p.d, p.Hq, p.T, p.B, p.q_sh, p.q_st, p.q_sb, G, kRows / G) ||
+      !make_map(&mk, p.kc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, kKeys) ||
+      !make_map(&mv, p.vc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, kKeys))
     return cudaErrorInvalidValue;
   const size_t smem = kSmemBytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_prefix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int ntiles = (p.T + p.node_tile - 1) / p.node_tile;
   dim3 grid(p.nchunk, ntiles, p.B * p.Hkv);
-  attn_prefix_tc_kernel<<<grid, kThreads, smem, stream>>>(maps.q, maps.k, maps.v, p);
+  attn_tc_kernel<<<grid, kThreads, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
 

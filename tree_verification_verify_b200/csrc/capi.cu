@@ -8,6 +8,7 @@
 
 namespace tv {
 size_t accept_workspace_bytes(int B, int T);
+constexpr int kAcceptMaxB = 16384;
 cudaError_t launch_accept(const tv_accept_args* a, int mode, void* ws, cudaStream_t stream);
 size_t expand_pool_bytes(int budget, int V);
 cudaError_t launch_expand_init(const tv_expand_args* a, int root_token, cudaStream_t stream);
@@ -90,9 +91,18 @@ AttnPlan plan_attn(const tv_attn_args* a) {
     pl.chunk_len = static_cast<int>(len);
     pl.nchunk = static_cast<int>((a->Lmax + len - 1) / len);
   }
+  if (pl.tc) {
+    // the merge uses one ticket per (sequence, kv head, row tile) group
+    const int64_t groups = static_cast<int64_t>(a->B) * a->Hkv * ntiles;
+    if (groups > kMaxTickets) { pl.nchunk = (a->Lmax > 0) ? 1 : 0; pl.chunk_len = a->Lmax > 0 ? ((a->Lmax + 127) / 128) * 128 : 128; }
+    if (pl.nchunk == 0) { pl.nchunk = 1; pl.chunk_len = 128; }
+  }
   const size_t rows = static_cast<size_t>(a->B) * a->T * a->Hq;
-  const size_t nparts = static_cast<size_t>(pl.nchunk) + 1;
-  size_t off = 0;
+  // the tensor-core path keeps a single chunk's result on chip; the other
+  // paths always merge (prefix chunks + the tree-path partial)
+  const size_t nparts = pl.tc ? (pl.nchunk > 1 ? static_cast<size_t>(pl.nchunk) : 0)
+                              : static_cast<size_t>(pl.nchunk) + 1;
+  size_t off = kTicketBytes;
   pl.off_o = off;  off = align256(off + nparts * rows * a->d * sizeof(float));
   pl.off_lse = off; off = align256(off + nparts * rows * sizeof(float));
   pl.off_ok = off;  off = align256(off + static_cast<size_t>(a->B) * a->T * sizeof(int32_t));
@@ -150,6 +160,7 @@ extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws
   p.part_o = reinterpret_cast<float*>(w + pl.off_o);
   p.part_lse = reinterpret_cast<float*>(w + pl.off_lse);
   p.node_ok = reinterpret_cast<int32_t*>(w + pl.off_ok);
+  p.tickets = reinterpret_cast<int32_t*>(w);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
   if (pl.sparse) {
@@ -165,7 +176,8 @@ extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws
     if (e != cudaSuccess) return from_cuda(e);
     e = launch_attn_sparse(p, s);
   } else if (pl.tc) {
-    e = launch_attn_tc(p, s);
+    // one kernel: prefix tiles, tree tiles and the split merge
+    return from_cuda(launch_attn_tc(p, s));
   } else {
     e = launch_attn_simt(p, s);
   }
@@ -188,6 +200,7 @@ int resolve_mode(const tv_accept_args* a) {
 tv_status check_accept(const tv_accept_args* a) {
   if (!a) return TV_ERR_INVALID_ARG;
   if (a->B < 0 || a->T < 0 || a->V < 1) return TV_ERR_INVALID_ARG;
+  if (a->B > kAcceptMaxB) return TV_ERR_UNSUPPORTED;
   if (a->mode < TV_ACCEPT_AUTO || a->mode > TV_ACCEPT_SPECEXEC) return TV_ERR_INVALID_ARG;
   if (!(a->temperature >= 0.f) || !std::isfinite(a->temperature)) return TV_ERR_INVALID_ARG;
   if (a->B > 0) {
