@@ -69,6 +69,9 @@ SHAPES = [
     (2, 33, 8, 1, 32, [77, 200], "fp32", "star"),
     (1, 15, 64, 8, 128, [2048], "bf16", "binary"),
     (2, 70, 16, 2, 128, [0, 700], "bf16", "recursive"),
+    (1, 300, 32, 8, 128, [200], "bf16", "chain"),        # deep: 3 gathered tree tiles
+    (2, 129, 8, 1, 128, [333, 1], "bf16", "binary"),
+    (1, 600, 64, 8, 128, [5000], "bf16", "recursive"),   # split prefix + fused merge
 ]
 
 
@@ -89,16 +92,17 @@ def test_shapes(shape):
     assert st == ref["status"] == 0
 
 
-def test_partial_trees_and_malformed_input():
+@pytest.mark.parametrize("L", [[250, 40, 3], [2500, 40, 3]], ids=["one-chunk", "split"])
+def test_partial_trees_and_malformed_input(L):
     T = 21
     par = tree_random_recursive(T, torch.Generator().manual_seed(2))
     par[13] = 17                                      # malformed: 17 >= 13
-    case = attn_case(3, T, 8, 2, 128, [250, 40, 3], "bf16", par, seed=5, n_nodes=[21, 9, 0])
+    case = attn_case(3, T, 8, 2, 128, L, "bf16", par, seed=5, n_nodes=[21, 9, 0])
     o, lse, _, st = _gpu(case)
     ref = _oracle(case)
     check_attn(o, ref, torch.bfloat16, lse_gpu=lse, poison=POISON)
     assert st == ref["status"] and st & ST_BAD_PARENT
-    bad_pl = torch.tensor([250, 999, 3], dtype=torch.int32)
+    bad_pl = torch.tensor([L[0], max(L) + 999, 3], dtype=torch.int32)
     bad_nn = torch.tensor([21, 9, 30], dtype=torch.int32)
     o, lse, _, st = _gpu(case, n_nodes=bad_nn, prefix_len=bad_pl)
     ref = _oracle(case, n_nodes=bad_nn, prefix_len=bad_pl)
