@@ -15,8 +15,7 @@
 // from parent[] (slot of node a in U = number of marked nodes below a in a
 // node bitmap).  All tiles share one online softmax.  With a single chunk
 // the CTA writes the final output; otherwise every chunk writes a partial
-// (O, lse) and the last CTA of the group (an atomic ticket, no waiting)
-// merges them.
+// (O, lse) and a merge kernel (one warp per output row) combines them.
 //
 // Warp roles (192 threads):
 //   warps 0-3  softmax / correction / epilogue: thread t owns query row t,
@@ -658,57 +657,64 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
-  if (p.nchunk == 1) return;
-  // ------------------------------------------------------------------ split merge
-  const int group = (b * p.Hkv + g) * gridDim.y + tile;
-  if (tid == 0) {
-    __threadfence();
-    const int done = atomicAdd(&p.tickets[group], 1);
-    bars.last = (done == p.nchunk - 1);
-  }
-  __syncthreads();
-  if (!bars.last || warp >= 4) return;
-  __threadfence();
-  // warp w merges rows 32w .. 32w+31; lane l first checks row 32w+l's path
-  const int myrow = warp * 32 + lane;
-  const bool mine_valid = (myrow / G) < nodes_here;
-  const bool mine_ok = mine_valid && path_ok(par, i0 + myrow / G);
+}
+
+// Log-sum-exp merge of the chunk partials of the tensor-core kernel: one
+// warp per (sequence, node, query head); lane c holds chunk c's lse, lane l
+// accumulates dimensions 4l .. 4l+3 with every chunk's load in flight.
+__global__ void __launch_bounds__(256) attn_tc_merge_kernel(AttnParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= static_cast<int64_t>(p.B) * p.T * p.Hq) return;
+  const int h = static_cast<int>(row % p.Hq);
+  const int i = static_cast<int>((row / p.Hq) % p.T);
+  const int b = static_cast<int>(row / (static_cast<int64_t>(p.Hq) * p.T));
+  const int n = p.n_nodes ? p.n_nodes[b] : p.T;
+  if (n < 0 || n > p.T || i >= n) return;
+  const int32_t* par = p.parent + b * p.par_sb;
+  const int L = p.prefix_len[b];
+  const bool bad_len = (L < 0 || L > p.Lmax);
+  const bool good = !bad_len && path_ok(par, i);
   const int np = p.nchunk;
-  for (int rr = 0; rr < 32; ++rr) {
-    const int r = warp * 32 + rr;
-    if (!__shfl_sync(0xffffffffu, mine_valid ? 1 : 0, rr)) continue;
-    const bool good = __shfl_sync(0xffffffffu, mine_ok ? 1 : 0, rr) && !bad_len;
-    const int node = i0 + r / G, head = g * G + r % G;
-    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + node * p.o_st + head * p.o_sh;
-    float lc = -INFINITY;
-    for (int c = lane; c < np; c += 32) lc = fmaxf(lc, __ldcg(&p.part_lse[part_row(p, c, b, node, head)]));
-    const float M = warp_max(lc);
-    const float wl = (lane < np && lc > -INFINITY) ? __expf(lc - M) : 0.f;
-    const float den = warp_sumf(wl);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = 0; c < np; ++c) {
-      const float w = __shfl_sync(0xffffffffu, wl, c & 31);
-      if (w == 0.f) continue;
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(p.part_o + part_row(p, c, b, node, head) * kD) + lane);
-      acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
-    }
-    const float inv = 1.f / den;
-    uint2 wv;
-    if (good && den > 0.f) {
-      wv.x = pack_bf16(acc.x * inv, acc.y * inv);
-      wv.y = pack_bf16(acc.z * inv, acc.w * inv);
-    } else {
-      wv.x = wv.y = pack_bf16(NAN, NAN);
-    }
-    *reinterpret_cast<uint2*>(o + lane * 4) = wv;
-    if (lane == 0) {
-      if (p.lse) p.lse[(static_cast<int64_t>(b) * p.T + node) * p.Hq + head] = (good && den > 0.f) ? M + __logf(den) : NAN;
-      if (!good && !bad_len) set_status(p.status, TV_DEV_BAD_PARENT);
-      if (bad_len && node == 0 && head == 0) set_status(p.status, TV_DEV_BAD_LEN);
+  float lc = -INFINITY;
+  if (lane < np) lc = __ldcg(&p.part_lse[part_row(p, lane, b, i, h)]);
+  const float M = warp_max(lc);
+  const float wl = (lane < np && lc > -INFINITY) ? __expf(lc - M) : 0.f;
+  const float den = warp_sumf(wl);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c0 = 0; c0 < np; c0 += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = (c0 + u < np) ? __ldcg(reinterpret_cast<const float4*>(p.part_o + part_row(p, c0 + u, b, i, h) * kD) + lane)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float w = __shfl_sync(0xffffffffu, wl, (c0 + u) & 31);
+      if (c0 + u < np) {
+        acc.x = fmaf(w, v[u].x, acc.x); acc.y = fmaf(w, v[u].y, acc.y);
+        acc.z = fmaf(w, v[u].z, acc.z); acc.w = fmaf(w, v[u].w, acc.w);
+      }
     }
   }
-  if (tid == 0) p.tickets[group] = 0;                // ready for the next call
+  const bool ok = good && den > 0.f;
+  const float inv = ok ? 1.f / den : 0.f;
+  uint2 wv;
+  if (ok) {
+    wv.x = pack_bf16(acc.x * inv, acc.y * inv);
+    wv.y = pack_bf16(acc.z * inv, acc.w * inv);
+  } else {
+    wv.x = wv.y = pack_bf16(NAN, NAN);
+  }
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + i * p.o_st + h * p.o_sh;
+  *reinterpret_cast<uint2*>(o + lane * 4) = wv;
+  if (lane == 0) {
+    if (p.lse) p.lse[row] = ok ? M + __logf(den) : NAN;
+    if (h == 0) {
+      if (!bad_len && !good) set_status(p.status, TV_DEV_BAD_PARENT);
+      if (bad_len && i == 0) set_status(p.status, TV_DEV_BAD_LEN);
+    }
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -791,6 +797,10 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream) {
   const int ntiles = (p.T + p.node_tile - 1) / p.node_tile;
   dim3 grid(p.nchunk, ntiles, p.B * p.Hkv);
   attn_tc_kernel<<<grid, kThreads, smem, stream>>>(mq, mk, mv, p);
+  if (p.nchunk > 1) {
+    const int64_t rows = static_cast<int64_t>(p.B) * p.T * p.Hq;
+    attn_tc_merge_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
+  }
   return cudaGetLastError();
 }
 
