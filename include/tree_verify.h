@@ -222,6 +222,25 @@ TV_API size_t tree_accept_workspace_size(const tv_accept_args* a);
 TV_API tv_status tree_accept(const tv_accept_args* a, void* ws, size_t ws_bytes,
                       tv_stream_t stream);
 
+/* tree_accept without a caller workspace (no counterpart in the paper; an
+ * interface addition of this library).  For callers that cannot allocate
+ * device memory: code whose device memory is owned by another runtime that
+ * reserved it up front (an inference server's pool), or code on a path
+ * where cudaMalloc's implicit device-wide synchronisation is not allowed.
+ * It computes exactly what tree_accept computes, with the same arguments.
+ * Scratch lives in a file-scope device array of the library, about 576 KB,
+ * held on every GPU that loads the library until the process exits; it is
+ * sized for B * T <= 32768 node rows and B <= 16384, and larger calls return
+ * TV_ERR_UNSUPPORTED.  The call allocates nothing (no cudaMalloc/cudaFree);
+ * it clears the counters it needs with cudaMemsetAsync on `stream`.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array and it keeps
+ * the last call's contents: calls that may overlap on the GPU (different
+ * streams, different host threads) race and must be serialised by the
+ * caller. */
+TV_API tv_status tree_accept_noalloc(const tv_accept_args* a, tv_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * tree_expand_topb
  *

@@ -20,7 +20,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["lib", "version", "status_string", "tree_verify_attn", "tree_accept",
+__all__ = ["lib", "version", "status_string", "tree_verify_attn", "tree_accept", "tree_accept_noalloc",
            "tree_expand_init", "tree_expand_topb", "ExpandState", "philox_uniforms",
            "TVError", "MODES"]
 
@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         for name, args in (("tree_verify_attn", [ctypes.POINTER(AttnArgs), c_vp, c_size, c_vp]),
                            ("tree_accept", [ctypes.POINTER(AcceptArgs), c_vp, c_size, c_vp]),
+                           ("tree_accept_noalloc", [ctypes.POINTER(AcceptArgs), c_vp]),
                            ("tree_expand_topb", [ctypes.POINTER(ExpandArgs), c_vp, c_size, c_vp]),
                            ("tree_expand_init", [ctypes.POINTER(ExpandArgs), c_i32, c_vp]),
                            ("tv_philox_uniforms", [c_u64, c_u64, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp])):
@@ -277,6 +278,44 @@ def tree_accept(target_logits, draft_tokens, parent, draft_probs=None, n_nodes=N
     sh = _stream(stream)
     ws = _workspace(dev, sh, need)
     _check(L.tree_accept(ctypes.byref(a), _aligned_ptr(ws), need, sh), "tree_accept")
+    return o
+
+
+def tree_accept_noalloc(target_logits, draft_tokens, parent, draft_probs=None, n_nodes=None,
+                        mode: str = "auto", temperature: float = 0.0, seed: int = 0, step: int = 0,
+                        dev_status=None, stream=None, outputs=None):
+    """tree_accept without a workspace, for callers that cannot allocate
+    device memory (include/tree_verify.h, tree_accept_noalloc): the library
+    uses a fixed scratch array of its own (B * T <= 32768).  Only the
+    outputs, when not given, are allocated here.  Calls that may overlap on
+    the GPU share that scratch and must be serialised by the caller."""
+    dev = _need_cuda(target_logits, draft_tokens, parent, draft_probs, n_nodes)
+    B, T, V = target_logits.shape
+    if target_logits.dtype != torch.float32 or target_logits.stride(-1) != 1:
+        raise TVError("target_logits must be fp32 with contiguous rows")
+    if draft_probs is not None and (draft_probs.dtype != torch.float32 or draft_probs.stride(-1) != 1):
+        raise TVError("draft_probs must be fp32 with contiguous rows")
+    for t in (draft_tokens, parent):
+        if t.dtype != torch.int32 or t.stride(-1) != 1:
+            raise TVError("draft_tokens / parent must be int32 with contiguous rows")
+    n_nodes = _i32(n_nodes)
+    if outputs is None:
+        outputs = dict(n_accepted=torch.empty(B, dtype=torch.int32, device=dev),
+                       accepted_nodes=torch.empty(B, T, dtype=torch.int32, device=dev),
+                       out_tokens=torch.empty(B, T + 1, dtype=torch.int32, device=dev),
+                       min_margin=torch.empty(B, dtype=torch.float64, device=dev))
+    o = outputs
+    dp = draft_probs
+    a = AcceptArgs(B, T, V,
+                   target_logits.data_ptr(), target_logits.stride(0), target_logits.stride(1),
+                   _ptr(dp), dp.stride(0) if dp is not None else 0, dp.stride(1) if dp is not None else 0,
+                   draft_tokens.data_ptr(), draft_tokens.stride(0),
+                   parent.data_ptr(), parent.stride(0),
+                   _ptr(n_nodes), MODES[mode], float(temperature),
+                   int(seed) & 0xFFFFFFFFFFFFFFFF, int(step) & 0xFFFFFFFFFFFFFFFF,
+                   o["n_accepted"].data_ptr(), o["accepted_nodes"].data_ptr(), o["out_tokens"].data_ptr(),
+                   _ptr(o.get("min_margin")), _ptr(dev_status))
+    _check(lib().tree_accept_noalloc(ctypes.byref(a), _stream(stream)), "tree_accept_noalloc")
     return o
 
 

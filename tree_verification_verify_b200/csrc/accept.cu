@@ -32,6 +32,8 @@
 // one segment only.
 #include <cooperative_groups.h>
 
+#include <mutex>
+
 #include "tv_common.cuh"
 
 namespace cg = cooperative_groups;
@@ -659,4 +661,50 @@ cudaError_t launch_accept(const tv_accept_args* a, int mode, void* ws, cudaStrea
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------ no-allocation entry
+
+int resolve_mode(const tv_accept_args* a);
+tv_status check_accept(const tv_accept_args* a);
+
+// Scratch of tree_accept_noalloc: the ticket region then the decisions of
+// at most kNoAllocMaxRows node rows.  Every GPU that loads the library holds
+// this array until the process exits.
+constexpr int kNoAllocMaxRows = 32768;
+constexpr size_t kNoAllocBytes = kAcceptTicketBytes + static_cast<size_t>(kNoAllocMaxRows) * sizeof(AcceptDec);
+static __device__ __align__(256) unsigned char g_accept_scratch[kNoAllocBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+}  // namespace
+
 }  // namespace tv
+
+// tree_accept for callers that cannot allocate device memory (see
+// include/tree_verify.h).  The first call on a device resolves the device
+// address of the file-scope scratch array with cudaGetSymbolAddress; later
+// calls reuse it.
+extern "C" tv_status tree_accept_noalloc(const tv_accept_args* a, tv_stream_t stream) {
+  using namespace tv;
+  const tv_status st = check_accept(a);
+  if (st != TV_OK) return st;
+  if (a->B == 0) return TV_OK;
+  if (static_cast<int64_t>(a->B) * a->T > kNoAllocMaxRows) return TV_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TV_ERR_CUDA;
+  void* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+      void* sym = nullptr;
+      if (cudaGetSymbolAddress(&sym, g_accept_scratch) != cudaSuccess || sym == nullptr) return TV_ERR_CUDA;
+      g_scratch_ptr[dev] = sym;
+    }
+    ptr = g_scratch_ptr[dev];
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the tickets must start at zero whatever an earlier call left behind
+  if (cudaMemsetAsync(ptr, 0, static_cast<size_t>(a->B) * sizeof(int32_t), s) != cudaSuccess) return TV_ERR_CUDA;
+  return launch_accept(a, resolve_mode(a), ptr, s) == cudaSuccess ? TV_OK : TV_ERR_CUDA;
+}

@@ -190,7 +190,7 @@ extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws
 
 // ------------------------------------------------------------ acceptance
 
-namespace {
+namespace tv {
 int resolve_mode(const tv_accept_args* a) {
   if (a->temperature == 0.f) return TV_ACCEPT_GREEDY;
   if (a->mode == TV_ACCEPT_AUTO) return TV_ACCEPT_SPECSAMPLE;
@@ -216,20 +216,20 @@ tv_status check_accept(const tv_accept_args* a) {
   }
   return TV_OK;
 }
-}  // namespace
+}  // namespace tv
 
 extern "C" size_t tree_accept_workspace_size(const tv_accept_args* a) {
-  if (check_accept(a) != TV_OK) return 0;
+  if (tv::check_accept(a) != TV_OK) return 0;
   return align256(accept_workspace_bytes(a->B, a->T));
 }
 
 extern "C" tv_status tree_accept(const tv_accept_args* a, void* ws, size_t ws_bytes,
                                  tv_stream_t stream) {
-  const tv_status st = check_accept(a);
+  const tv_status st = tv::check_accept(a);
   if (st != TV_OK) return st;
   if (a->B == 0) return TV_OK;
   if (!ws_ok(ws, ws_bytes, accept_workspace_bytes(a->B, a->T))) return TV_ERR_WORKSPACE;
-  return from_cuda(launch_accept(a, resolve_mode(a), ws, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_accept(a, tv::resolve_mode(a), ws, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 // ------------------------------------------------------------ expansion
