@@ -14,9 +14,10 @@
 // finish (an atomic ticket, no waiting) walks the decisions from the root.
 //
 // Layout of a row pass.  A thread-block cluster of C CTAs (C <= 8) owns one
-// node row; CTA rank r owns a contiguous slice of 128-element segments.  A
-// warp owns a segment at a time (lane l holds elements 4l..4l+3, one 16-byte
-// load) and keeps kUnroll segments in flight.  Cross-CTA sums and maxima go
+// node row; CTA rank r owns a contiguous slice of 512-element segments.  A
+// warp owns a segment at a time: four warp-wide 16-byte loads, lane l holding
+// elements 128k + 4l .. 128k + 4l + 3 (k = 0..3); full segments are read
+// without bounds checks.  Cross-CTA sums and maxima go
 // through distributed shared memory (double-buffered slots, one cluster
 // barrier per reduction); every CTA computes the same reduced values and so
 // takes the same branches.
@@ -32,6 +33,7 @@
 // one segment only.
 #include <cooperative_groups.h>
 
+#include <cfloat>
 #include <mutex>
 
 #include "tv_common.cuh"
@@ -66,14 +68,14 @@ struct AcceptParams {
   int32_t* out_tokens;
   double* min_margin;
   int C;                    // CTAs per row (cluster size)
-  int seg_per_cta;          // 128-element segments per CTA
+  int seg_per_cta;          // 512-element segments per CTA
 };
 
 constexpr int kAcceptThreads = 256;
 constexpr int kAcceptWarps = kAcceptThreads / kWarp;
-constexpr int kSeg = 128;
-constexpr int kUnroll = 4;
-constexpr int kMaxSegPerCta = 512;      // 65536 elements per CTA
+constexpr int kSeg = 512;               // elements per segment
+constexpr int kSub = 128;               // elements of one warp-wide float4 load
+constexpr int kMaxSegPerCta = 128;      // 65536 elements per CTA
 
 // ------------------------------------------------------------ shared state
 
@@ -168,39 +170,46 @@ struct Frame {
   bool resid;
 };
 
+// The four float4 of segment start s0 held by this lane (elements
+// s0 + 128k + 4l ..); positions past the row end read `fill`.
+__device__ __forceinline__ void load_seg(const float* __restrict__ row, int s0, int V, bool vec, float fill,
+                                         float4 (&v)[4]) {
+  const int lane = threadIdx.x & 31;
+  if (vec && s0 + kSeg <= V) {
+    const float4* p = reinterpret_cast<const float4*>(row + s0) + lane;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = __ldg(p + 32 * k);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = load4(row, s0 + k * kSub + 4 * lane, V, vec, fill);
+  }
+}
+
 // One pass over this CTA's slice: segment sums of the current weights into
-// seg_out; returns the slice total (fp64).
+// seg_out; returns the slice total (fp64).  Past the row end the logits read
+// -FLT_MAX, whose weight is 0.
 template <bool READQ>
 __device__ double weight_pass(const float* zr, const float* qr, bool zvec, bool qvec, int V, int seg0, int nloc,
                               const Frame& f, float* seg_out, AcceptShared& sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   double tot = 0.0;
-  for (int base = warp; base < nloc; base += kAcceptWarps * kUnroll) {
-    float4 zv[kUnroll], qv[kUnroll];
+  for (int s = warp; s < nloc; s += kAcceptWarps) {
+    const int s0 = (seg0 + s) * kSeg;
+    float4 zv[4], qv[4];
+    load_seg(zr, s0, V, zvec, -FLT_MAX, zv);
+    if (READQ) load_seg(qr, s0, V, qvec, 0.f, qv);
+    float g = 0.f;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int s = base + u * kAcceptWarps;
-      if (s < nloc) {
-        const int e0 = (seg0 + s) * kSeg + lane * 4;
-        zv[u] = load4(zr, e0, V, zvec, -INFINITY);
-        if (READQ) qv[u] = load4(qr, e0, V, qvec, 0.f);
-        else qv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+    for (int k = 0; k < 4; ++k) {
+      const float4 q4 = READQ ? qv[k] : make_float4(0.f, 0.f, 0.f, 0.f);
+      g += weight(zv[k].x, q4.x, f.k, f.zoff, f.inv_s, f.c, f.resid);
+      g += weight(zv[k].y, q4.y, f.k, f.zoff, f.inv_s, f.c, f.resid);
+      g += weight(zv[k].z, q4.z, f.k, f.zoff, f.inv_s, f.c, f.resid);
+      g += weight(zv[k].w, q4.w, f.k, f.zoff, f.inv_s, f.c, f.resid);
     }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int s = base + u * kAcceptWarps;
-      if (s < nloc) {
-        // fill values (-inf logits) give weight 0 past the row end
-        float g = weight(zv[u].x, qv[u].x, f.k, f.zoff, f.inv_s, f.c, f.resid);
-        g += weight(zv[u].y, qv[u].y, f.k, f.zoff, f.inv_s, f.c, f.resid);
-        g += weight(zv[u].z, qv[u].z, f.k, f.zoff, f.inv_s, f.c, f.resid);
-        g += weight(zv[u].w, qv[u].w, f.k, f.zoff, f.inv_s, f.c, f.resid);
-        const float ss = warp_sum_f(g);
-        if (lane == 0) seg_out[s] = ss;
-        tot += static_cast<double>(ss);
-      }
-    }
+    const float ss = warp_sum_f(g);
+    if (lane == 0) seg_out[s] = ss;
+    tot += static_cast<double>(ss);
   }
   return block_sum_d(lane == 0 ? tot : 0.0, sh);
 }
@@ -247,46 +256,60 @@ __device__ void slice_search(const float* zr, const float* qr, bool zvec, bool q
     seg = __shfl_sync(0xffffffffu, last, L);
     if (seg < 0) seg = 0;
   }
-  const int e0 = (seg0 + seg) * kSeg + lane * 4;
-  const float4 zv = load4(zr, e0, V, zvec, -INFINITY);
-  float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (f.resid) qv = load4(qr, e0, V, qvec, 0.f);
-  double w[4];
-  w[0] = weight(zv.x, qv.x, f.k, f.zoff, f.inv_s, f.c, f.resid);
-  w[1] = weight(zv.y, qv.y, f.k, f.zoff, f.inv_s, f.c, f.resid);
-  w[2] = weight(zv.z, qv.z, f.k, f.zoff, f.inv_s, f.c, f.resid);
-  w[3] = weight(zv.w, qv.w, f.k, f.zoff, f.inv_s, f.c, f.resid);
+  const int s0 = (seg0 + seg) * kSeg;
+  float4 zv[4], qv[4];
+  load_seg(zr, s0, V, zvec, -FLT_MAX, zv);
+  if (f.resid) load_seg(qr, s0, V, qvec, 0.f, qv);
+  else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) qv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   int t = -1;
   double margin = 0.0;
-  if (found) {
-    const double lsum = ((w[0] + w[1]) + w[2]) + w[3];
-    const double li = cb + warp_incl_scan(lsum);
-    double le = __shfl_up_sync(0xffffffffu, li, 1);
-    if (lane == 0) le = cb;
-    const unsigned m2 = __ballot_sync(0xffffffffu, li > target);
-    if (m2 != 0u) {
-      const int L = __ffs(m2) - 1;
-      if (lane == L) {
-        double cum = le;
-        for (int k = 0; k < 4; ++k) {
-          if (cum + w[k] > target) {
-            t = e0 + k;
-            margin = fmin(cum + w[k] - target, target - cum) / W;
-            break;
+  int lastpos = -1;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int e0 = s0 + k * kSub + lane * 4;
+    double w[4];
+    w[0] = weight(zv[k].x, qv[k].x, f.k, f.zoff, f.inv_s, f.c, f.resid);
+    w[1] = weight(zv[k].y, qv[k].y, f.k, f.zoff, f.inv_s, f.c, f.resid);
+    w[2] = weight(zv[k].z, qv[k].z, f.k, f.zoff, f.inv_s, f.c, f.resid);
+    w[3] = weight(zv[k].w, qv[k].w, f.k, f.zoff, f.inv_s, f.c, f.resid);
+    for (int e = 0; e < 4; ++e) if (w[e] > 0.0 && e0 + e < V) lastpos = e0 + e;
+    if (found && t < 0) {
+      const double lsum = ((w[0] + w[1]) + w[2]) + w[3];
+      const double li = cb + warp_incl_scan(lsum);
+      double le = __shfl_up_sync(0xffffffffu, li, 1);
+      if (lane == 0) le = cb;
+      const unsigned m2 = __ballot_sync(0xffffffffu, li > target);
+      if (m2 != 0u) {
+        const int L = __ffs(m2) - 1;
+        int tt = -1;
+        double mg = 0.0;
+        if (lane == L) {
+          double cum = le;
+          for (int e = 0; e < 4; ++e) {
+            if (cum + w[e] > target) {
+              tt = e0 + e;
+              mg = fmin(cum + w[e] - target, target - cum) / W;
+              break;
+            }
+            cum += w[e];
           }
-          cum += w[k];
         }
+        t = __shfl_sync(0xffffffffu, tt, L);
+        margin = __shfl_sync(0xffffffffu, mg, L);
       }
-      t = __shfl_sync(0xffffffffu, t, L);
-      margin = __shfl_sync(0xffffffffu, margin, L);
+      cb = __shfl_sync(0xffffffffu, li, 31);
     }
   }
   if (t < 0) {
-    int lp = -1;
-    for (int k = 0; k < 4; ++k) if (w[k] > 0.0 && e0 + k < V) lp = e0 + k;
-    const unsigned mm = __ballot_sync(0xffffffffu, lp >= 0);
-    const int L = mm ? 31 - __clz(mm) : 0;
-    t = __shfl_sync(0xffffffffu, lp, L);
+    // rounding put the crossing past this segment: its last positive element
+    const unsigned mm = __ballot_sync(0xffffffffu, lastpos >= 0);
+    int best = lastpos;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+    t = mm ? best : s0;
     margin = 0.0;
   }
   *out_t = t;
@@ -398,41 +421,43 @@ accept_node_kernel(AcceptParams p) {
   float bv = -INFINITY;
   int bi = INT_MAX;
   bool bad = false;
-  for (int base = warp; base < nloc; base += kAcceptWarps * kUnroll) {
-    float4 v[kUnroll], qv[kUnroll];
+  float nf = 0.f;                 // x * 0 turns any non-finite x into NaN
+  float qmin = 0.f;
+  for (int s = warp; s < nloc; s += kAcceptWarps) {
+    const int s0 = (seg0 + s) * kSeg;
+    float4 v[4], qv[4];
+    load_seg(zr, s0, V, zvec, greedy ? -INFINITY : -FLT_MAX, v);
+    if (read_q) load_seg(qr, s0, V, qvec, 0.f, qv);
+    if (greedy) {
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int s = base + u * kAcceptWarps;
-      if (s < nloc) {
-        const int e0 = (seg0 + s) * kSeg + lane * 4;
-        v[u] = load4(zr, e0, V, zvec, -INFINITY);
-        if (read_q) qv[u] = load4(qr, e0, V, qvec, 0.f);
-      }
-    }
+      for (int k = 0; k < 4; ++k) {
+        const int e0 = s0 + k * kSub + lane * 4;
+        const float xs[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int s = base + u * kAcceptWarps;
-      if (s < nloc) {
-        const int e0 = (seg0 + s) * kSeg + lane * 4;
-        const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int idx = e0 + k;
-          if (idx < V) {
-            const float x = xs[k];
-            if (greedy ? isnan(x) : !isfinite(x)) bad = true;
-            else if (x > bv || (x == bv && idx < bi)) { bv = x; bi = idx; }
+        for (int e = 0; e < 4; ++e) {
+          const float x = xs[e];
+          if (e0 + e < V) {
+            if (x != x) bad = true;
+            else if (x > bv || (x == bv && e0 + e < bi)) { bv = x; bi = e0 + e; }
           }
         }
-        if (read_q) {
-          const float qs[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
+      }
+    } else {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            if (e0 + k < V && !(qs[k] >= 0.f && isfinite(qs[k]))) bad = true;
+      for (int k = 0; k < 4; ++k) {
+        bv = fmaxf(fmaxf(bv, v[k].x), fmaxf(v[k].y, fmaxf(v[k].z, v[k].w)));
+        nf = fmaf(v[k].x, 0.f, nf); nf = fmaf(v[k].y, 0.f, nf);
+        nf = fmaf(v[k].z, 0.f, nf); nf = fmaf(v[k].w, 0.f, nf);
+        if (read_q) {
+          qmin = fminf(qmin, fminf(fminf(qv[k].x, qv[k].y), fminf(qv[k].z, qv[k].w)));
+          nf = fmaf(qv[k].x, 0.f, nf); nf = fmaf(qv[k].y, 0.f, nf);
+          nf = fmaf(qv[k].z, 0.f, nf); nf = fmaf(qv[k].w, 0.f, nf);
         }
       }
     }
   }
+  if (!greedy && (nf != nf || qmin < 0.f)) bad = true;
+  if (!greedy) bi = 0;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -637,7 +662,7 @@ cudaError_t launch_accept(const tv_accept_args* a, int mode, void* ws, cudaStrea
   p.min_margin = a->min_margin;
   if (a->B == 0) return cudaSuccess;
   const int nseg = (a->V + kSeg - 1) / kSeg;
-  int C = (nseg + 127) / 128;                  // ~16k elements per CTA
+  int C = (nseg + 31) / 32;                    // ~16k elements per CTA
   if (C < 1) C = 1;
   if (C > 8) C = 8;
   p.C = C;
