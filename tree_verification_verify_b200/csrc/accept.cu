@@ -661,13 +661,20 @@ cudaError_t launch_accept(const tv_accept_args* a, int mode, void* ws, cudaStrea
   p.n_acc = a->n_accepted; p.acc_nodes = a->accepted_nodes; p.out_tokens = a->out_tokens;
   p.min_margin = a->min_margin;
   if (a->B == 0) return cudaSuccess;
+  // CTAs per row: few rows need several CTAs per row (the sampling modes
+  // make sequential passes over a row); many rows already fill the GPU and
+  // extra CTAs only add cluster synchronisation.  The sampling modes keep
+  // per-segment sums in shared memory, which bounds the slice length.
   const int nseg = (a->V + kSeg - 1) / kSeg;
-  int C = (nseg + 31) / 32;                    // ~16k elements per CTA
-  if (C < 1) C = 1;
-  if (C > 8) C = 8;
+  const int64_t rows_total = static_cast<int64_t>(a->B) * (a->T > 0 ? a->T : 1);
+  int C;
+  if (mode == TV_ACCEPT_GREEDY) C = rows_total >= 256 ? 1 : (rows_total >= 64 ? 2 : 4);
+  else C = rows_total >= 256 ? 2 : 4;
+  if (mode != TV_ACCEPT_GREEDY) C = max(C, (nseg + kMaxSegPerCta - 1) / kMaxSegPerCta);
+  C = min(C, max(1, nseg));
+  if (C > 8) return cudaErrorInvalidValue;
   p.C = C;
   p.seg_per_cta = (nseg + C - 1) / C;
-  if (p.seg_per_cta > kMaxSegPerCta) return cudaErrorInvalidValue;
   const int rows = a->T > 0 ? a->T : 1;        // T == 0: one cluster writes the empty result
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rows * C, a->B, 1);

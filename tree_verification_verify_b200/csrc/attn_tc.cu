@@ -429,8 +429,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       bool ok = true;
+      // the tree tiles follow the prefix tiles; their count is known once the
+      // producer has built the union of root paths
       int ntot = nprefix;
-      if (has_tree) {
+      if (has_tree && nprefix == 0) {
         ok = mbar_wait(&bars.tree_info, 0, abort);
         ntot += (bars.nU + kKeys - 1) / kKeys;
       }
@@ -450,7 +452,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         }
         mma_commit(&bars.s_full[0]);
       }
+      bool tree_known = !has_tree || nprefix == 0;
       for (int j = 0; j < ntot && ok; ++j) {
+        if (!tree_known && j + 1 == ntot) {
+          ok = mbar_wait(&bars.tree_info, 0, abort);
+          if (!ok) break;
+          ntot += (bars.nU + kKeys - 1) / kKeys;
+          tree_known = true;
+        }
         if (j + 1 < ntot) {
           const int s1 = (j + 1) % kStages;
           ok = mbar_wait(&bars.full[s1], ((j + 1) / kStages) & 1, abort);
@@ -490,12 +499,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     bool ok = true;
     int ntot = nprefix;
     bool my_ok = true;
-    if (has_tree) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars.tree_info, 0, abort));
-      ntot += (bars.nU + kKeys - 1) / kKeys;
-      my_ok = row_valid && bars.node_ok[tid / G] != 0;
-    }
-    for (int j = 0; j < ntot && ok; ++j) {
+    bool tree_known = !has_tree;
+    for (int j = 0; ok; ++j) {
+      if (!tree_known && j == nprefix) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars.tree_info, 0, abort));
+        if (!ok) break;
+        ntot += (bars.nU + kKeys - 1) / kKeys;
+        my_ok = row_valid && bars.node_ok[tid / G] != 0;
+        tree_known = true;
+      }
+      if (j >= ntot) break;
       const bool tree_tile = j >= nprefix;
       const int nk = tree_tile ? 0 : min(kKeys, k1 - (k0 + j * kKeys));
       uint32_t mk[4] = {0u, 0u, 0u, 0u};
@@ -634,7 +647,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
-        if (row_valid) p.part_lse[part_row(p, chunk, b, row_node, row_head)] = lse;
+        if (row_valid) {
+          // invalid rows carry NaN into the merge
+          const bool good = my_ok && !bad_len;
+          p.part_lse[part_row(p, chunk, b, row_node, row_head)] = good ? lse : NAN;
+          if (has_tree && !my_ok) set_status(p.status, TV_DEV_BAD_PARENT);
+          if (bad_len && chunk == 0 && row_node == 0 && row_head == 0) set_status(p.status, TV_DEV_BAD_LEN);
+        }
       }
     }
   }
@@ -661,7 +680,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
 
 // Log-sum-exp merge of the chunk partials of the tensor-core kernel: one
 // warp per (sequence, node, query head); lane c holds chunk c's lse, lane l
-// accumulates dimensions 4l .. 4l+3 with every chunk's load in flight.
+// accumulates dimensions 4l .. 4l+3 with every chunk's load in flight.  The
+// partials of rows that are invalid (malformed parent chain, prefix length
+// out of range) carry lse = NaN and the merged row is NaN.
 __global__ void __launch_bounds__(256) attn_tc_merge_kernel(AttnParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -671,13 +692,12 @@ __global__ void __launch_bounds__(256) attn_tc_merge_kernel(AttnParams p) {
   const int b = static_cast<int>(row / (static_cast<int64_t>(p.Hq) * p.T));
   const int n = p.n_nodes ? p.n_nodes[b] : p.T;
   if (n < 0 || n > p.T || i >= n) return;
-  const int32_t* par = p.parent + b * p.par_sb;
-  const int L = p.prefix_len[b];
-  const bool bad_len = (L < 0 || L > p.Lmax);
-  const bool good = !bad_len && path_ok(par, i);
+  // a NaN partial lse marks a row the tensor-core kernel found invalid
   const int np = p.nchunk;
   float lc = -INFINITY;
   if (lane < np) lc = __ldcg(&p.part_lse[part_row(p, lane, b, i, h)]);
+  const bool good = !__any_sync(0xffffffffu, lc != lc);
+  if (!good) lc = -INFINITY;
   const float M = warp_max(lc);
   const float wl = (lane < np && lc > -INFINITY) ? __expf(lc - M) : 0.f;
   const float den = warp_sumf(wl);
@@ -708,13 +728,7 @@ __global__ void __launch_bounds__(256) attn_tc_merge_kernel(AttnParams p) {
   }
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + i * p.o_st + h * p.o_sh;
   *reinterpret_cast<uint2*>(o + lane * 4) = wv;
-  if (lane == 0) {
-    if (p.lse) p.lse[row] = ok ? M + __logf(den) : NAN;
-    if (h == 0) {
-      if (!bad_len && !good) set_status(p.status, TV_DEV_BAD_PARENT);
-      if (bad_len && i == 0) set_status(p.status, TV_DEV_BAD_LEN);
-    }
-  }
+  if (lane == 0 && p.lse) p.lse[row] = ok ? M + __logf(den) : NAN;
 }
 
 // ------------------------------------------------------------------ host side
