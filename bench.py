@@ -158,21 +158,46 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 
 class Step:
-    """Device-resident inputs of one workload and the calls of one step."""
+    """Device-resident inputs of one workload and the calls of one step.
+
+    The SpecExec-shaped workload builds its 2048-node tree on the device in
+    every step (16 best-first rounds of 128 from N(0, 4^2) draft logits over
+    32000 tokens), then verifies it (attention over that tree) and accepts
+    with SpecExec's rule at temperature 0.6."""
 
     def __init__(self, name, seed, dev):
         import tree_verification_verify_b200 as tv
-        from synth import CONFIGS, config_attn_case, config_accept_case, tree_depths
+        from synth import CONFIGS, config_attn_case, config_accept_case, config_expand_case, tree_depths
         self.tv = tv
         self.name = name
         base = "longctx" if name == "longctx_sparse" else name
         self.c = c = CONFIGS[base]
         self.sparse = name == "longctx_sparse"
         self.dev = dev
+        self.expand = None
         self.attn = config_attn_case(base, seed=seed, device=dev, sparse=self.sparse)
         temp = c.get("temperature", c.get("temperatures", (0.0,))[-1])
-        self.acc = config_accept_case(base, temperature=temp, seed=seed, device=dev,
-                                      parents=[p.cpu().numpy() for p in self.attn.parent])
+        if base == "specexec70b":
+            ec = config_expand_case(base, seed=seed)
+            self.ec = ec
+            self.exp_state = tv.tree_expand_init(ec.budget, ec.V, ec.Bsel, device=dev)
+            calls = ec.n_calls()
+            self.exp_logits = [ec.round_logits(k, 1 if k == 0 else ec.Bsel, device=dev) for k in range(calls)]
+            self.exp_root = torch.zeros(1, dtype=torch.int32, device=dev)
+            self.run_expand()
+            torch.cuda.synchronize()
+            par = self.exp_state.parent.view(1, -1)
+            tok = self.exp_state.token.view(1, -1)
+            self.attn.parent = par
+            self.acc = config_accept_case(base, temperature=temp, seed=seed, device=dev,
+                                          parents=[par[0].cpu().numpy()], mode="specexec")
+            self.acc.parent = par
+            self.acc.draft_tokens = tok
+            self.acc.mode = "specexec"
+            self.expand = True
+        else:
+            self.acc = config_accept_case(base, temperature=temp, seed=seed, device=dev,
+                                          parents=[p.cpu().numpy() for p in self.attn.parent])
         self.temperature = temp
         B, T, Hq, d = self.attn.q.shape
         self.B, self.T = B, T
@@ -204,6 +229,16 @@ class Step:
             for b in range(B):
                 internal += len(set(par[b][1:].tolist()))
         self.accept_bytes = float(B * T * V * 4 + internal * V * 4)
+        self.expand_bytes = 0.0
+        if self.expand:
+            self.expand_bytes = float(sum(x.numel() for x in self.exp_logits) * 4)
+
+    def run_expand(self):
+        tv, st, ec = self.tv, self.exp_state, self.ec
+        tv.tree_expand_init(ec.budget, ec.V, ec.Bsel, state=st)
+        for k, z in enumerate(self.exp_logits):
+            rows = self.exp_root if k == 0 else st.frontier
+            tv.tree_expand_topb(st, z, rows)
 
     def run_attn(self):
         a = self.attn
@@ -214,59 +249,68 @@ class Step:
     def run_accept(self):
         c = self.acc
         self.tv.tree_accept(c.target_logits, c.draft_tokens, c.parent, draft_probs=c.draft_probs,
-                            temperature=self.temperature, seed=c.seed, step=0, dev_status=self.status,
-                            outputs=self.acc_out)
+                            mode=c.mode, temperature=self.temperature, seed=c.seed, step=0,
+                            dev_status=self.status, outputs=self.acc_out)
 
     def launches_per_step(self):
-        return (5 if self.sparse else 3) + 2
+        attn = self.attn_launches
+        exp = (1 + 2 * len(self.exp_logits)) if self.expand else 0
+        return attn + 1 + exp
 
 
 def capture_graphs(step):
-    """CUDA graphs of the two calls of a step (captured once, replayed in
-    the timed region so that no host launch overhead sits between kernels)."""
+    """CUDA graphs of the calls of a step (captured once, replayed in the
+    timed region so that no host launch overhead sits between kernels)."""
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         for _ in range(2):                       # warm the library's host-side setup
+            if step.expand:
+                step.run_expand()
             step.run_attn()
             step.run_accept()
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
+    step.attn_path = step.tv.last_attn_path
+    step.attn_launches = step.tv.last_attn_launches
     # capture on the warm-up stream: the binding's per-stream workspace then
     # already exists and nothing is allocated (or zero-filled) in the graph
-    g_attn, g_acc = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_attn, stream=s):
-        step.run_attn()
-    with torch.cuda.graph(g_acc, stream=s):
-        step.run_accept()
+    graphs = {}
+    for name, fn in (("expand", step.run_expand if step.expand else None),
+                     ("attn", step.run_attn), ("accept", step.run_accept)):
+        if fn is None:
+            continue
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            fn()
+        graphs[name] = g
     torch.cuda.synchronize()
-    return g_attn, g_acc
+    return graphs
 
 
 def time_steps(step, K, W, world, flush):
-    g_attn, g_acc = capture_graphs(step)
+    graphs = capture_graphs(step)
+    names = list(graphs)
     s = torch.cuda.current_stream()
     for _ in range(W):
         flush.zero_()
-        g_attn.replay()
-        g_acc.replay()
+        for nm in names:
+            graphs[nm].replay()
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize()
     for k in range(K):
         flush.zero_()
         ev[k][0].record(s)
-        g_attn.replay()
-        ev[k][1].record(s)
-        g_acc.replay()
-        ev[k][2].record(s)
+        for j, nm in enumerate(names):
+            graphs[nm].replay()
+            ev[k][j + 1].record(s)
     torch.cuda.synchronize()
     barrier(world)
-    t_attn = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
-    t_acc = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
-    del g_attn, g_acc
-    return t_attn, t_acc
+    times = {nm: [ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(K)] for j, nm in enumerate(names)}
+    del graphs
+    return times
 
 
 def time_e2e(step, K, W, flush):
@@ -274,8 +318,11 @@ def time_e2e(step, K, W, flush):
     step's inputs are copied host->device and the accepted tokens read
     back inside the timed region."""
     a, c = step.attn, step.acc
-    dev_in = [a.q, a.k_cache, a.v_cache, a.prefix_len, a.k_tree, a.v_tree, a.parent,
-              c.target_logits, c.draft_tokens]
+    dev_in = [a.q, a.k_cache, a.v_cache, a.prefix_len, a.k_tree, a.v_tree, c.target_logits]
+    if step.expand:
+        dev_in += step.exp_logits          # the tree itself is built on the device
+    else:
+        dev_in += [a.parent, c.draft_tokens]
     if c.draft_probs is not None:
         dev_in.append(c.draft_probs)
     host_in = [t.cpu().pin_memory() for t in dev_in]
@@ -288,6 +335,8 @@ def time_e2e(step, K, W, flush):
     def one():
         for d, h in zip(dev_in, host_in):
             d.copy_(h, non_blocking=True)
+        if step.expand:
+            step.run_expand()
         step.run_attn()
         step.run_accept()
         host_out[0].copy_(step.acc_out["n_accepted"], non_blocking=True)
@@ -330,8 +379,26 @@ def cpu_baseline(step, budget_s=15.0):
     ch = dict(z=c.target_logits.cpu(), q=None if c.draft_probs is None else c.draft_probs.cpu(),
               tok=c.draft_tokens.cpu(), par=c.parent.cpu())
     t0 = time.perf_counter()
-    o_accept(ch["z"], ch["q"], ch["tok"], ch["par"], temperature=step.temperature, seed=c.seed)
+    o_accept(ch["z"], ch["q"], ch["tok"], ch["par"], mode=c.mode, temperature=step.temperature, seed=c.seed)
     t_acc = time.perf_counter() - t0
+    t_exp, exp_note = 0.0, ""
+    if step.expand:
+        # expansion: the first calls of the build (all 16 take about as long
+        # as each other past the first), scaled to the whole build
+        from oracle.expand import ExpandState as OState, expand_call
+        ec = step.ec
+        ost = OState(ec.budget, ec.root_token)
+        frontier = [0]
+        n_calls, done_calls, t_e = len(step.exp_logits), 0, 0.0
+        while done_calls < min(3, n_calls):
+            z = step.exp_logits[done_calls].cpu().double().numpy()
+            t0 = time.perf_counter()
+            frontier = list(expand_call(ost, z[:len(frontier)] if done_calls else z[:1],
+                                        np.asarray(frontier, np.int64), ec.Bsel))
+            t_e += time.perf_counter() - t0
+            done_calls += 1
+        t_exp = t_e / done_calls * n_calls
+        exp_note = f", plus {done_calls} of {n_calls} expansion rounds scaled to the build"
     B, T = step.B, step.T
     done = 0
     t_attn = 0.0
@@ -344,11 +411,11 @@ def cpu_baseline(step, budget_s=15.0):
         t_attn += time.perf_counter() - t0
         done += 1
     per_node = t_attn / done
-    t_step = per_node * B * T + t_acc
+    t_step = per_node * B * T + t_acc + t_exp
     return {"value": (B * T) / t_step, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
             "sample": f"attention of {done} of {B * T} nodes (all heads, fp64) scaled to the step, "
-                      f"plus the full acceptance walk ({t_acc:.2f} s)",
-            "seconds": round(t_attn + t_acc, 2)}
+                      f"plus the full acceptance walk ({t_acc:.2f} s){exp_note}",
+            "seconds": round(t_attn + t_acc + t_exp, 2)}
 
 
 # --------------------------------------------------------------------------
@@ -414,19 +481,25 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     clk = ClockSampler(local)
     clk.start()
-    t_attn, t_acc = time_steps(step, args.steps, args.warmup, world, flush)
+    times = time_steps(step, args.steps, args.warmup, world, flush)
     clocks = clk.stop()
-    ms_step = statistics.fmean([a + b for a, b in zip(t_attn, t_acc)])
-    ms_step = max_over_ranks(ms_step, world)
-    ms_attn = max_over_ranks(statistics.fmean(t_attn), world)
-    ms_acc = max_over_ranks(statistics.fmean(t_acc), world)
+    per_step = [sum(ts) for ts in zip(*times.values())]
+    ms_step = max_over_ranks(statistics.fmean(per_step), world)
+    ms_attn = max_over_ranks(statistics.fmean(times["attn"]), world)
+    ms_acc = max_over_ranks(statistics.fmean(times["accept"]), world)
+    ms_exp = max_over_ranks(statistics.fmean(times["expand"]), world) if "expand" in times else 0.0
     e2e_ms, h2d, d2h = time_e2e(step, max(3, args.steps // 5), 3, flush)
     e2e_ms = max_over_ranks(e2e_ms, world)
     tokens = step.B * step.T * world
     hbm, bf16, bf16_sus, src = peaks()
     # dominant call and its roofline
     attn_t = max(step.attn_bytes / (hbm * 1e9), step.attn_flops / (bf16 * 1e12))
-    if ms_acc >= ms_attn:
+    if ms_exp >= max(ms_acc, ms_attn):
+        achieved = step.expand_bytes / (ms_exp * 1e-3) / 1e9
+        roof = {"kernel": "tree_expand_topb (16 rounds: row + merge launches)", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                "traffic": None, "peak_source": src, "algorithmic_bytes": step.expand_bytes}
+    elif ms_acc >= ms_attn:
         achieved = step.accept_bytes / (ms_acc * 1e-3) / 1e9
         roof = {"kernel": "tree_accept (node + walk launches)", "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
@@ -453,11 +526,15 @@ def main():
                   "attn_tflops": round(step.attn_flops / (ms_attn * 1e-3) / 1e12, 2),
                   "accept_gbs": round(step.accept_bytes / (ms_acc * 1e-3) / 1e9, 1),
                   "accept_nodes_per_s": step.B * step.T / (ms_acc * 1e-3)},
+        "launches_per_step": step.launches_per_step(),
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": step.launches_per_step() * args.steps,
         "clocks": clocks,
     }
+    if step.expand:
+        line["calls"]["tree_expand_us"] = round(ms_exp * 1e3, 2)
+        line["calls"]["expand_gbs"] = round(step.expand_bytes / (ms_exp * 1e-3) / 1e9, 1)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(step)
     if rank == 0:

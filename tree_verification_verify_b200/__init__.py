@@ -103,6 +103,8 @@ def lib() -> ctypes.CDLL:
             f.restype = c_size
         L.tv_attn_path.argtypes = [ctypes.POINTER(AttnArgs)]
         L.tv_attn_path.restype = c_i32
+        L.tv_attn_launches.argtypes = [ctypes.POINTER(AttnArgs)]
+        L.tv_attn_launches.restype = c_i32
         L.tree_expand_pool_bytes.argtypes = [c_i32, c_i32]
         L.tree_expand_pool_bytes.restype = c_size
         L.tree_verify_version.restype = ctypes.c_char_p
@@ -224,8 +226,9 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent, n_
                  out.data_ptr(), out.stride(0), out.stride(1), out.stride(2),
                  _ptr(lse), _ptr(sel_blocks), _ptr(dev_status))
     L = lib()
-    global last_attn_path
+    global last_attn_path, last_attn_launches
     last_attn_path = L.tv_attn_path(ctypes.byref(a))
+    last_attn_launches = L.tv_attn_launches(ctypes.byref(a))
     need = L.tree_verify_attn_workspace_size(ctypes.byref(a))
     sh = _stream(stream)
     ws = _workspace(dev, sh, need)
@@ -235,6 +238,7 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent, n_
 
 # Which attention kernels the last tree_verify_attn call ran (tv_attn_path).
 last_attn_path = None
+last_attn_launches = None
 ATTN_PATHS = {0: "cuda-core split-KV", 1: "tcgen05 prefix", 2: "block top-k sparse"}
 
 

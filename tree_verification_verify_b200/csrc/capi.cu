@@ -133,6 +133,15 @@ extern "C" int32_t tv_attn_path(const tv_attn_args* a) {
   return pl.sparse ? 2 : (pl.tc ? 1 : 0);
 }
 
+extern "C" int32_t tv_attn_launches(const tv_attn_args* a) {
+  if (check_attn(a) != TV_OK) return -1;
+  if (a->B == 0 || a->T == 0) return 0;
+  const AttnPlan pl = plan_attn(a);
+  if (pl.sparse) return (a->k_block_mean ? 0 : 1) + 4;
+  if (pl.tc) return pl.nchunk > 1 ? 2 : 1;
+  return 3;
+}
+
 extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws_bytes,
                                       tv_stream_t stream) {
   const tv_status st = check_attn(a);
