@@ -298,8 +298,8 @@ TV_API tv_status tree_expand_topb(const tv_expand_args* a, void* ws, size_t ws_b
 TV_API int32_t tv_attn_path(const tv_attn_args* a);
 /* How many kernels tree_verify_attn launches for these arguments (0 when
  * B or T is 0, -1 when the arguments are rejected): 1 for the tensor-core
- * kernel with the whole prefix in one chunk, 2 when its chunk partials are
- * merged, 3 on the CUDA-core path (prefix, tree paths, merge), 4 or 5 on
+ * kernel (its prefix chunks are merged inside the launch), 3 on the
+ * CUDA-core path (prefix, tree paths, merge), 4 or 5 on
  * the block top-k path (block means unless the caller passes them, block
  * selection, sparse prefix, tree paths, merge).  Host only; nothing runs. */
 TV_API int32_t tv_attn_launches(const tv_attn_args* a);

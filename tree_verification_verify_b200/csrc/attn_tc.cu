@@ -8,72 +8,92 @@
 // is loaded once for all nodes and heads of the tile (the "inter-draft-token
 // reuse" of the sparse verification page, "Methodology" 4).
 //
-// One CTA owns (sequence, kv head, 128-row tile, prefix chunk).  Its key
-// tiles are the chunk's prefix tiles of 128 keys and, in chunk 0, the tree
-// tiles: the union U of the tile's nodes' root paths, gathered into K/V
-// tiles and masked per row by an ancestor bitmask built in shared memory
-// from parent[] (slot of node a in U = number of marked nodes below a in a
-// node bitmap).  All tiles share one online softmax.  With a single chunk
-// the CTA writes the final output; otherwise every chunk writes a partial
-// (O, lse) and a merge kernel (one warp per output row) combines them.
+// One CTA owns (sequence, kv head, 128-row tile, prefix chunk); the chunks
+// of one row tile form a thread-block cluster.  A CTA's key tiles are its
+// chunk's prefix tiles of 128 keys and, in the last chunk, the tree tiles: the
+// union U of the tile's nodes' root paths, gathered into K/V tiles and
+// masked per row by the row's ancestors in U.  All tiles share one online
+// softmax.  At the end every CTA pushes its normalised O rows and their
+// log-sum-exp over distributed shared memory to the CTA of the cluster that
+// merges them; each CTA merges a share of the rows and writes the output.
 //
-// Warp roles (192 threads):
+// Warp roles (256 threads):
 //   warps 0-3  softmax / correction / epilogue: thread t owns query row t,
 //              which is TMEM lane t (tcgen05.ld 32x32b);
-//   warp 4     producer: Q once, prefix K/V tiles by TMA into a two-stage
-//              ring (128B-swizzled; K-major for K, MN-major for V), the
-//              tree bookkeeping, and the gathered tree tiles (cp.async);
-//   warp 5     TMEM allocator and MMA issuer (one thread): S = Q K^T into one
-//              of two TMEM S buffers, O += P V into the TMEM O accumulator.
-// Online softmax in base 2 with a lazily updated row maximum: O and the row
-// sum are rescaled only when the maximum grows by more than 2^8, which keeps
-// P <= 256 (exact in the final O / l).  P goes to shared memory as bf16 in
-// the 128B-swizzled K-major layout the PV MMA reads.
+//   warp 4     Q and the K tiles: TMA into a three-stage ring (128B swizzle,
+//              K-major) or, for tree tiles, a cp.async gather;
+//   warp 5     TMEM allocator and MMA issuer (one thread): S = Q K^T into
+//              one of two TMEM S buffers, O += P V with P read from TMEM;
+//   warp 6     the V tiles, a two-stage ring (MN-major), like warp 4;
+//   warp 7     tree bookkeeping (last chunk): parent[] into shared memory,
+//              the node bitmap of U, the slot of every node of U and the
+//              slot of its parent.
+// A K stage is released when its S = Q K^T completes, a V stage when its
+// P V completes, so the loads of later tiles start while earlier tiles are
+// in the softmax.  Online softmax in base 2 with a lazily updated row
+// maximum: O and the row sum are rescaled only when the maximum grows by
+// more than 2^8, which keeps P <= 256 (exact in the final O / l).  P is
+// written as bf16 over the first 64 columns of its S buffer.
 //
 // Every mbarrier wait is bounded: on expiry the CTA records TV_DEV_TIMEOUT,
-// stops issuing work, drains what it issued and frees its TMEM.
+// stops issuing work, drains what it issued, frees its TMEM, and its rows
+// come out as NaN.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cooperative_groups.h>
 
 #include "attn.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace tv {
 
 namespace tc {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;
+constexpr int kWarpK = 4, kWarpMma = 5, kWarpV = 6, kWarpTree = 7;
 constexpr int kRows = 128;          // M
 constexpr int kKeys = 128;          // keys per tile (N of QK, K of PV)
 constexpr int kD = 128;
-constexpr int kStages = 2;
+constexpr int kKS = 3;              // K ring stages
+constexpr int kVS = 2;              // V ring stages
 constexpr int kMaxT = 4096;         // tree nodes handled by this kernel
+constexpr int kMaxCluster = 8;      // chunks per row tile
 constexpr uint32_t kHalfBytes = kRows * 128;            // 128 rows x 128 B
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;         // 32 KB (d = 128 bf16)
 constexpr uint32_t kSmemQ = 0;
-constexpr uint32_t kSmemKV = kSmemQ + kTileBytes;       // stage s: K at +s*64K, V at +32K
-constexpr uint32_t kSmemP = kSmemKV + kStages * 2 * kTileBytes;
-constexpr uint32_t kSmemU = kSmemP + kTileBytes;        // U list (int32, kMaxT)
-constexpr uint32_t kSmemBytes = kSmemU + kMaxT * 4;     // 208 KB
-constexpr uint32_t kTmemCols = 512;                     // S0, S1, O (128 each)
+constexpr uint32_t kSmemK = kSmemQ + kTileBytes;
+constexpr uint32_t kSmemV = kSmemK + kKS * kTileBytes;
+constexpr uint32_t kSmemPar = kSmemV + kVS * kTileBytes;  // parent[] (u16)
+constexpr uint32_t kSmemUL = kSmemPar + kMaxT * 2;        // U: slot -> node (u16)
+constexpr uint32_t kSmemUP = kSmemUL + kMaxT * 2;         // U: slot -> parent's slot (u16)
+constexpr uint32_t kSmemBytes = kSmemUP + kMaxT * 2;      // 216 KB
+constexpr uint32_t kSmemInbox = kSmemK;                   // merge: fp32 O rows pushed by the cluster
+constexpr uint32_t kTmemCols = 512;                       // S0, S1, O (128 each)
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint32_t kDrainLimit = 1u << 20;
+constexpr uint16_t kRootMark = 0xFFFEu;   // parent[] entry of a well-formed root
+constexpr uint16_t kBadMark = 0xFFFFu;    // malformed parent (or no parent slot)
+
+static_assert(kSmemInbox + (kRows + kMaxCluster) * kD * 4 <= kSmemK + kKS * kTileBytes,
+              "the merge inbox fits the K ring");
 
 struct Bars {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
   uint64_t q_full;
-  uint64_t s_full[2];
-  uint64_t s_free[2];
-  uint64_t p_full;
+  uint64_t k_full[kKS], k_empty[kKS];
+  uint64_t v_full[kVS], v_empty[kVS];
+  uint64_t s_full[2], p_full[2];
   uint64_t pv_done;
   uint64_t tree_info;
   uint32_t tmem_base;
   int abort;
   int nU;                           // nodes in the union of root paths
-  int last;                         // this CTA merges the group
   uint32_t bm[kMaxT / 32];          // node bitmap of U
   int pre[kMaxT / 32];              // marked nodes below each bitmap word
   int node_ok[kRows];               // root path of the tile's node is well formed
+  float in_lse[kRows + kMaxCluster]; // merge inbox: log2-sum-exp of row (chunk, row)
+  int in_abort[kMaxCluster];        // merge inbox: the chunk's CTA aborted
 };
 
 
@@ -206,35 +226,52 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+// D (TMEM) (+)= A (TMEM, K-major: row m in lane m, two bf16 per column) x B
+// (shared memory descriptor).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Wait used while draining after an abort: bounded, ignores the abort flag.
+__device__ __forceinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
+  const uint32_t a = smem_u32(b);
+  for (uint32_t it = 0; it < kDrainLimit; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return;
+  }
+}
+
 // Slot of node a in U: the number of marked nodes below a.
 __device__ __forceinline__ int u_slot(const Bars& bars, int a) {
   return bars.pre[a >> 5] + __popc(bars.bm[a >> 5] & ((1u << (a & 31)) - 1u));
 }
 
-// Ancestor bitmask of node i (whose root path is well formed) over tree
-// tile tt, i.e. the slots [128 tt, 128 tt + 128) of U.
-__device__ __forceinline__ void tree_mask(const int32_t* par, int i, int tt, const Bars& bars, uint32_t* mk) {
-  mk[0] = mk[1] = mk[2] = mk[3] = 0u;
-  int j = i;
-  for (int step = 0; step <= i; ++step) {
-    const int sl = u_slot(bars, j);
-    if ((sl >> 7) == tt) mk[(sl >> 5) & 3] |= 1u << (sl & 31);
-    if (j == 0) break;
-    j = par[j];
-  }
-}
-
-// Whether node i's root path reaches node 0 through parent[j] in [0, j).
-__device__ __forceinline__ bool path_ok(const int32_t* par, int i) {
-  if (par[0] != -1) return false;
-  int j = i;
-  for (int step = 0; step <= i && j != 0; ++step) {
-    const int pj = par[j];
-    if (pj < 0 || pj >= j) return false;
-    j = pj;
-  }
-  return true;
-}
+__device__ __forceinline__ uint32_t s_col(int j) { return (j & 1) ? kColS1 : kColS0; }
 
 }  // namespace tc
 
@@ -245,14 +282,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                const __grid_constant__ CUtensorMap tmap_v, AttnParams p) {
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ Bars bars;
-  const int chunk = blockIdx.x;
+  cg::cluster_group cl = cg::this_cluster();
+  const int chunk = blockIdx.x;            // = rank in the cluster (the cluster spans the chunks)
+  const int C = static_cast<int>(gridDim.x);
   const int tile = blockIdx.y;
   const int b = blockIdx.z / p.Hkv, g = blockIdx.z % p.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.G;
+  // the early exits depend on (sequence, row tile) only: a cluster leaves whole
   const int n = p.n_nodes ? p.n_nodes[b] : p.T;
   if (n < 0 || n > p.T) {
-    if (chunk == 0 && tile == 0 && g == 0 && tid == 0) set_status(p.status, TV_DEV_BAD_LEN);
+    if (chunk == C - 1 && tile == 0 && g == 0 && tid == 0) set_status(p.status, TV_DEV_BAD_LEN);
     return;
   }
   const int i0 = tile * (kRows / G);
@@ -265,32 +305,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   const int k1 = min(k0 + p.chunk_len, L);
   const int nprefix = (k1 > k0) ? (k1 - k0 + kKeys - 1) / kKeys : 0;
   const int nodes_here = min(kRows / G, n - i0);
+  const bool has_tree = (chunk == C - 1);   // the last chunk is the shortest
   // this thread's query row (softmax warps)
   const int row_node = i0 + tid / G;
-  const int row_head = g * G + tid % G;
   const bool row_valid = tid < kRows && (tid / G) < nodes_here;
 
   // 1024-aligned dynamic shared memory (128B swizzle atoms are 1 KB)
   const uint32_t raw = smem_u32(dsmem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = dsmem_raw + (base - raw);
-  int* ulist = reinterpret_cast<int*>(gbase + kSmemU);
+  uint16_t* spar = reinterpret_cast<uint16_t*>(gbase + kSmemPar);
+  uint16_t* ulist = reinterpret_cast<uint16_t*>(gbase + kSmemUL);
+  uint16_t* uparent = reinterpret_cast<uint16_t*>(gbase + kSmemUP);
   volatile int* abort = &bars.abort;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&bars.full[s], 1); mbar_init(&bars.empty[s], 1); }
     mbar_init(&bars.q_full, 1);
-    for (int s = 0; s < 2; ++s) { mbar_init(&bars.s_full[s], 1); mbar_init(&bars.s_free[s], 4); }
-    mbar_init(&bars.p_full, 4);
+    for (int s = 0; s < kKS; ++s) { mbar_init(&bars.k_full[s], 1); mbar_init(&bars.k_empty[s], 1); }
+    for (int s = 0; s < kVS; ++s) { mbar_init(&bars.v_full[s], 1); mbar_init(&bars.v_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&bars.s_full[s], 1); mbar_init(&bars.p_full[s], 4); }
     mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.tree_info, 1);
     bars.abort = 0;
     bars.nU = 0;
-    bars.last = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&bars.tmem_base)),
                  "r"(kTmemCols)
@@ -301,47 +342,36 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   __syncthreads();
   fence_after();
   const uint32_t tmem = bars.tmem_base;
-  const bool has_tree = (chunk == 0);
+  float orow[kD];              // softmax threads: this row's normalised O
+  float my_lse2 = NAN;         // and its log2-sum-exp
 
-  if (warp == 4) {
-    // ---------------------------------------------------------------- producer
-    const int first = min(nprefix, kStages);
-    if (lane == 0) {
-      const uint32_t sq = base + kSmemQ;
-      mbar_expect_tx(&bars.q_full, kTileBytes);
-      tma_load_4d(&tmap_q, sq, &bars.q_full, 0, g * G, i0, b);
-      tma_load_4d(&tmap_q, sq + kHalfBytes, &bars.q_full, 64, g * G, i0, b);
-      for (int j = 0; j < first; ++j) {
-        const uint32_t sk = base + kSmemKV + j * 2 * kTileBytes;
-        const int kb = k0 + j * kKeys;
-        mbar_expect_tx(&bars.full[j], 2 * kTileBytes);
-        tma_load_4d(&tmap_k, sk, &bars.full[j], 0, g, kb, b);
-        tma_load_4d(&tmap_k, sk + kHalfBytes, &bars.full[j], 64, g, kb, b);
-        tma_load_4d(&tmap_v, sk + kTileBytes, &bars.full[j], 0, g, kb, b);
-        tma_load_4d(&tmap_v, sk + kTileBytes + kHalfBytes, &bars.full[j], 64, g, kb, b);
-      }
-    }
-    int ntree = 0;
+  if (warp == kWarpTree) {
+    // ------------------------------------------------------------ tree bookkeeping
     if (has_tree) {
-      // union U of the root paths of this tile's nodes, as a node bitmap
+      for (int j = lane; j < n; j += 32) {
+        const int pj = par[j];
+        spar[j] = (j == 0) ? (pj == -1 ? kRootMark : kBadMark)
+                           : ((pj >= 0 && pj < j) ? static_cast<uint16_t>(pj) : kBadMark);
+      }
       const int nw = (n + 31) >> 5;
       for (int w = lane; w < nw; w += 32) bars.bm[w] = 0u;
       __syncwarp();
+      // mark the root path of every node of the tile (parents strictly
+      // decrease, so a walk takes at most i + 1 steps)
       for (int r = lane; r < nodes_here; r += 32) {
-        const int i = i0 + r;
-        int ok = (par[0] == -1) ? 1 : 0;
-        int j = i;
-        for (int step = 0; step <= i; ++step) {
+        int j = i0 + r;
+        int ok = 1;
+        for (int step = 0; step <= i0 + r; ++step) {
           atomicOr(&bars.bm[j >> 5], 1u << (j & 31));
-          if (j == 0) break;
-          const int pj = par[j];
-          if (pj < 0 || pj >= j) { ok = 0; break; }
+          const uint16_t pj = spar[j];
+          if (pj == kRootMark) break;
+          if (pj == kBadMark) { ok = 0; break; }
           j = pj;
         }
         bars.node_ok[r] = ok;
       }
       __syncwarp();
-      // prefix counts per bitmap word, then the U list in node order
+      // prefix counts per bitmap word, then U in node order
       const int per = (nw + 31) / 32;
       const int lo = min(lane * per, nw), hi = min(lo + per, nw);
       int cnt = 0;
@@ -358,179 +388,235 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         uint32_t m = bars.bm[w];
         while (m) {
           const int bit = __ffs(m) - 1;
-          ulist[run++] = w * 32 + bit;
+          ulist[run++] = static_cast<uint16_t>(w * 32 + bit);
           m &= m - 1u;
         }
       }
-      if (lane == 31) bars.nU = incl;
+      const int nU = __shfl_sync(0xffffffffu, incl, 31);
       __syncwarp();
-      ntree = (bars.nU + kKeys - 1) / kKeys;
+      // the parent of a node of U is in U (or the node is the root / malformed)
+      for (int sl = lane; sl < nU; sl += 32) {
+        const uint16_t pa = spar[ulist[sl]];
+        uparent[sl] = (pa < kRootMark) ? static_cast<uint16_t>(u_slot(bars, pa)) : kBadMark;
+      }
+      if (lane == 0) bars.nU = nU;
+      __syncwarp();
       if (lane == 0) mbar_arrive(&bars.tree_info);
     }
-    const int ntot = nprefix + ntree;
-    int issued = first;
-    for (int j = first; j < ntot; ++j) {
-      const int s = j % kStages;
-      bool ok = true;
-      if (j >= kStages) {
+  } else if (warp == kWarpK || warp == kWarpV) {
+    // ------------------------------------------------------------ producers
+    const bool isk = (warp == kWarpK);
+    const int NS = isk ? kKS : kVS;
+    uint64_t* full = isk ? bars.k_full : bars.v_full;
+    uint64_t* empty = isk ? bars.k_empty : bars.v_empty;
+    const CUtensorMap* map = isk ? &tmap_k : &tmap_v;
+    const uint32_t ring = base + (isk ? kSmemK : kSmemV);
+    const __nv_bfloat16* src_tree = static_cast<const __nv_bfloat16*>(isk ? p.kt : p.vt);
+    if (isk && lane == 0) {
+      const uint32_t sq = base + kSmemQ;
+      mbar_expect_tx(&bars.q_full, kTileBytes);
+      tma_load_4d(&tmap_q, sq, &bars.q_full, 0, g * G, i0, b);
+      tma_load_4d(&tmap_q, sq + kHalfBytes, &bars.q_full, 64, g * G, i0, b);
+    }
+    int ntot = nprefix, ntree = 0;
+    bool tree_known = !has_tree;
+    int issued = 0;
+    for (int j = 0;; ++j) {
+      if (!tree_known && j == nprefix) {
         bool w = true;
-        if (lane == 0) w = mbar_wait(&bars.empty[s], ((j / kStages) - 1) & 1, abort);
-        ok = __all_sync(0xffffffffu, w);
+        if (lane == 0) w = mbar_wait(&bars.tree_info, 0, abort);
+        if (!__all_sync(0xffffffffu, w)) break;
+        ntree = (bars.nU + kKeys - 1) / kKeys;
+        ntot += ntree;
+        tree_known = true;
       }
-      if (!ok) break;
-      const uint32_t sk = base + kSmemKV + s * 2 * kTileBytes;
+      if (j >= ntot) break;
+      const int s = j % NS;
+      if (j >= NS) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&empty[s], ((j / NS) - 1) & 1, abort);
+        if (!__all_sync(0xffffffffu, w)) break;
+      }
+      const uint32_t dst = ring + s * kTileBytes;
       if (j < nprefix) {
         if (lane == 0) {
           const int kb = k0 + j * kKeys;
-          mbar_expect_tx(&bars.full[s], 2 * kTileBytes);
-          tma_load_4d(&tmap_k, sk, &bars.full[s], 0, g, kb, b);
-          tma_load_4d(&tmap_k, sk + kHalfBytes, &bars.full[s], 64, g, kb, b);
-          tma_load_4d(&tmap_v, sk + kTileBytes, &bars.full[s], 0, g, kb, b);
-          tma_load_4d(&tmap_v, sk + kTileBytes + kHalfBytes, &bars.full[s], 64, g, kb, b);
+          mbar_expect_tx(&full[s], kTileBytes);
+          tma_load_4d(map, dst, &full[s], 0, g, kb, b);
+          tma_load_4d(map, dst + kHalfBytes, &full[s], 64, g, kb, b);
         }
       } else {
-        // gathered tree tile: rows = U[128 tt ..], 128B-swizzled like TMA writes
-        const int tt = j - nprefix;
+        // gathered tree tile (tree tiles run from the last slots down):
+        // rows = U[128 tt ..], 128B-swizzled as TMA writes them
+        const int tt = ntree - 1 - (j - nprefix);
         const int nU = bars.nU;
-        const __nv_bfloat16* kt = static_cast<const __nv_bfloat16*>(p.kt);
-        const __nv_bfloat16* vt = static_cast<const __nv_bfloat16*>(p.vt);
+        uint8_t* gdst = gbase + (dst - base);
         for (int e = lane; e < kRows * 16; e += 32) {
           const int r = e >> 4, c = e & 15;
           const int slot = tt * kKeys + r;
           const uint32_t off = static_cast<uint32_t>(c >> 3) * kHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
           if (slot < nU) {
             const int a = ulist[slot];
-            const int64_t src = b * p.kt_sb + static_cast<int64_t>(a) * p.kt_st + g * p.kt_sh + c * 8;
-            cp_async16(sk + off, kt + src);
-            cp_async16(sk + kTileBytes + off, vt + src);
+            cp_async16(dst + off, src_tree + b * p.kt_sb + static_cast<int64_t>(a) * p.kt_st + g * p.kt_sh + c * 8);
           } else {
-            *reinterpret_cast<uint4*>(gbase + (sk - base) + off) = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(gbase + (sk - base) + kTileBytes + off) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(gdst + off) = make_uint4(0u, 0u, 0u, 0u);
           }
         }
         cp_async_wait_all();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.full[s]);
+        if (lane == 0) mbar_arrive(&full[s]);
       }
       ++issued;
     }
-    // drain: every issued load must land before the CTA can exit
+    // drain: every issued load lands before the CTA can exit
     if (lane == 0) {
-      mbar_wait(&bars.q_full, 0, abort);
-      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
-        uint32_t it = 0;
-        while (!mbar_wait(&bars.full[j % kStages], (j / kStages) & 1, abort) && ++it < 4) {
-        }
-      }
+      if (isk) mbar_drain(&bars.q_full, 0);
+      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j) mbar_drain(&full[j % NS], (j / NS) & 1);
     }
     __syncwarp();
-  } else if (warp == 5) {
-    // ---------------------------------------------------------------- MMA issuer
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      bool ok = true;
-      // the tree tiles follow the prefix tiles; their count is known once the
-      // producer has built the union of root paths
       int ntot = nprefix;
-      if (has_tree && nprefix == 0) {
-        ok = mbar_wait(&bars.tree_info, 0, abort);
-        ntot += (bars.nU + kKeys - 1) / kKeys;
-      }
-      const uint32_t idesc_qk = instr_desc(kRows, kKeys, 0, 0);
-      const uint32_t idesc_pv = instr_desc(kRows, kD, 0, 1);
-      const uint32_t sq = base + kSmemQ, sp = base + kSmemP;
-      if (ok && ntot > 0) ok = mbar_wait(&bars.q_full, 0, abort);
-      if (ok && ntot > 0) ok = mbar_wait(&bars.full[0], 0, abort);
-      if (ok && ntot > 0) {
-        fence_after();
-        const uint32_t sk = base + kSmemKV;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_bf16(tmem + kColS0, smem_desc(sq + off, 16, 1024), smem_desc(sk + off, 16, 1024), idesc_qk,
-                   kk > 0);
-        }
-        mma_commit(&bars.s_full[0]);
-      }
-      bool tree_known = !has_tree || nprefix == 0;
-      for (int j = 0; j < ntot && ok; ++j) {
-        if (!tree_known && j + 1 == ntot) {
-          ok = mbar_wait(&bars.tree_info, 0, abort);
-          if (!ok) break;
+      bool tree_known = !has_tree;
+      bool ok = true;
+      // the tree tiles follow the prefix tiles; their count is known once
+      // the tree warp has built U
+      auto know = [&](int upto) -> bool {
+        if (!tree_known && upto >= nprefix) {
+          if (!mbar_wait(&bars.tree_info, 0, abort)) return false;
           ntot += (bars.nU + kKeys - 1) / kKeys;
           tree_known = true;
         }
-        if (j + 1 < ntot) {
-          const int s1 = (j + 1) % kStages;
-          ok = mbar_wait(&bars.full[s1], ((j + 1) / kStages) & 1, abort);
-          if (ok && j >= 1) ok = mbar_wait(&bars.s_free[(j + 1) & 1], ((j - 1) >> 1) & 1, abort);
-          if (!ok) break;
-          fence_after();
-          const uint32_t sk = base + kSmemKV + s1 * 2 * kTileBytes;
-          const uint32_t dcol = ((j + 1) & 1) ? kColS1 : kColS0;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            mma_bf16(tmem + dcol, smem_desc(sq + off, 16, 1024), smem_desc(sk + off, 16, 1024), idesc_qk,
-                     kk > 0);
-          }
-          mma_commit(&bars.s_full[(j + 1) & 1]);
-        }
-        ok = mbar_wait(&bars.p_full, j & 1, abort);
-        if (!ok) break;
-        fence_after();
-        const uint32_t sv = base + kSmemKV + (j % kStages) * 2 * kTileBytes + kTileBytes;
+        return true;
+      };
+      const uint32_t idesc_qk = instr_desc(kRows, kKeys, 0, 0);
+      const uint32_t idesc_pv = instr_desc(kRows, kD, 0, 1);
+      const uint32_t sq = base + kSmemQ;
+      int s_issued = 0, pv_issued = 0;
+      auto issue_s = [&](int j) {
+        const uint32_t sk = base + kSmemK + (j % kKS) * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_bf16(tmem + kColO, smem_desc(sp + aoff, 16, 1024), smem_desc(sv + kk * 2048, kHalfBytes, 1024),
-                   idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          mma_bf16(tmem + s_col(j), smem_desc(sq + off, 16, 1024), smem_desc(sk + off, 16, 1024), idesc_qk,
+                   kk > 0);
         }
+        mma_commit(&bars.k_empty[j % kKS]);
+        mma_commit(&bars.s_full[j & 1]);
+        ++s_issued;
+      };
+      ok = know(0);
+      if (ok && ntot > 0) ok = mbar_wait(&bars.q_full, 0, abort);
+      for (int j = 0; j < 2 && ok; ++j) {
+        ok = know(j);
+        if (!ok || j >= ntot) break;
+        ok = mbar_wait(&bars.k_full[j % kKS], (j / kKS) & 1, abort);
+        if (!ok) break;
+        fence_after();
+        issue_s(j);
+      }
+      for (int j = 0; ok; ++j) {
+        ok = know(j);
+        if (!ok || j >= ntot) break;
+        ok = mbar_wait(&bars.p_full[j & 1], (j >> 1) & 1, abort);
+        if (ok) ok = mbar_wait(&bars.v_full[j % kVS], (j / kVS) & 1, abort);
+        if (!ok) break;
+        fence_after();
+        const uint32_t sv = base + kSmemV + (j % kVS) * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + kColO, tmem + s_col(j) + kk * 8, smem_desc(sv + kk * 2048, kHalfBytes, 1024),
+                      idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars.v_empty[j % kVS]);
         mma_commit(&bars.pv_done);
-        mma_commit(&bars.empty[j % kStages]);
+        ++pv_issued;
+        const int jn = j + 2;
+        ok = know(jn);
+        if (!ok) break;
+        if (jn < ntot) {
+          ok = mbar_wait(&bars.k_full[jn % kKS], (jn / kKS) & 1, abort);
+          // S(jn) overwrites the buffer P(j) is read from
+          if (ok) ok = mbar_wait(&bars.pv_done, j & 1, abort);
+          if (!ok) break;
+          fence_after();
+          issue_s(jn);
+        }
+      }
+      if (!ok) {
+        // the issued MMAs complete before the TMEM is freed
+        if (s_issued > 0) mbar_drain(&bars.s_full[(s_issued - 1) & 1], ((s_issued - 1) >> 1) & 1);
+        if (pv_issued > 0) mbar_drain(&bars.pv_done, (pv_issued - 1) & 1);
       }
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- softmax warps 0-3
+    // ------------------------------------------------------------ softmax warps 0-3
     const float sl2 = p.scale * 1.4426950408889634f;   // scores in log2 units
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    int ntot = nprefix;
+    int ntot = nprefix, ntree = 0;
     bool my_ok = true;
     bool tree_known = !has_tree;
+    int cur = -1;                 // walk position (slot) on this row's root path
     for (int j = 0; ok; ++j) {
       if (!tree_known && j == nprefix) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bars.tree_info, 0, abort));
         if (!ok) break;
-        ntot += (bars.nU + kKeys - 1) / kKeys;
+        ntree = (bars.nU + kKeys - 1) / kKeys;
+        ntot += ntree;
         my_ok = row_valid && bars.node_ok[tid / G] != 0;
+        cur = my_ok ? u_slot(bars, row_node) : -1;
         tree_known = true;
       }
       if (j >= ntot) break;
       const bool tree_tile = j >= nprefix;
       const int nk = tree_tile ? 0 : min(kKeys, k1 - (k0 + j * kKeys));
-      uint32_t mk[4] = {0u, 0u, 0u, 0u};
-      if (tree_tile && my_ok) tree_mask(par, row_node, j - nprefix, bars, mk);
+      // key mask of the tile: four words, kept in registers
+      uint32_t mk0 = 0u, mk1 = 0u, mk2 = 0u, mk3 = 0u;
+      if (tree_tile) {
+        // ancestors of this row's node in slots [128 tt, 128 tt + 128); the
+        // tiles run downwards and slots decrease along the path, so the walk
+        // continues where the previous tile left it
+        const int lo = (ntree - 1 - (j - nprefix)) * kKeys;
+        while (cur >= lo) {
+          if (cur < lo + kKeys) {
+            const int w = (cur - lo) >> 5;
+            const uint32_t bit = 1u << (cur & 31);
+            mk0 |= (w == 0) ? bit : 0u;
+            mk1 |= (w == 1) ? bit : 0u;
+            mk2 |= (w == 2) ? bit : 0u;
+            mk3 |= (w == 3) ? bit : 0u;
+          }
+          const uint16_t up = uparent[cur];
+          cur = (up == kBadMark) ? -1 : static_cast<int>(up);
+        }
+      } else {
+        mk0 = nk >= 32 ? 0xffffffffu : ((1u << nk) - 1u);
+        mk1 = nk >= 64 ? 0xffffffffu : (nk <= 32 ? 0u : ((1u << (nk - 32)) - 1u));
+        mk2 = nk >= 96 ? 0xffffffffu : (nk <= 64 ? 0u : ((1u << (nk - 64)) - 1u));
+        mk3 = nk >= 128 ? 0xffffffffu : (nk <= 96 ? 0u : ((1u << (nk - 96)) - 1u));
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full[j & 1], (j >> 1) & 1, abort));
       if (!ok) break;
       fence_after();
       float s[kKeys];
-      const uint32_t scol = (j & 1) ? kColS1 : kColS0;
+      const uint32_t scol = s_col(j);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(trow + scol + c * 32, s + c * 32);
       tmem_wait_ld();
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.s_free[j & 1]);
-      float mt = -INFINITY;
+      // masked scores in log2 units; the maximum over four interleaved
+      // partial maxima (the maximum does not depend on the order)
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int c = 0; c < kKeys; ++c) {
-        const bool keep = tree_tile ? ((mk[c >> 5] >> (c & 31)) & 1u) != 0u : c < nk;
-        s[c] = keep ? s[c] * sl2 : -INFINITY;
-        mt = fmaxf(mt, s[c]);
+        const uint32_t mw = (c < 32) ? mk0 : (c < 64) ? mk1 : (c < 96) ? mk2 : mk3;
+        s[c] = ((mw >> (c & 31)) & 1u) ? s[c] * sl2 : -INFINITY;
+        mx[c & 3] = fmaxf(mx[c & 3], s[c]);
       }
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const float m_new = fmaxf(m_run, mt);
       const bool first = (j == 0);
       const bool grow = !first && (m_new > m_run + 8.0f);
@@ -542,36 +628,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         m_run = m_new;
       }
       const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-      float rs = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < kKeys; ++c) {
         s[c] = ex2_approx(s[c] - mu);
-        rs += s[c];
+        ps[c & 3] += s[c];
       }
-      l_run = l_run * factor + rs;
-      if (j > 0) {
+      l_run = l_run * factor + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+      if (__any_sync(0xffffffffu, grow)) {
+        // O holds the tiles up to j - 1: wait for their P V, then rescale
         ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (j - 1) & 1, abort));
         if (!ok) break;
         fence_after();
-        if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float o[32];
-            tmem_ld32(trow + kColO + c * 32, o);
-            tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(trow + kColO + c * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= factor;
-            tmem_st32(trow + kColO + c * 32, o);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) o[e] *= factor;
+          tmem_st32(trow + kColO + c * 32, o);
         }
       }
+      // P as bf16 pairs over the first 64 columns of the S buffer
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(s[64 * h + 2 * e], s[64 * h + 2 * e + 1]);
+        tmem_st32u(trow + scol + 32 * h, pk);
+      }
+      tmem_wait_st();
       if (!tree_tile && nk < kKeys) {
         // ragged prefix tile: V rows past the prefix end may hold anything
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars.full[j % kStages], (j / kStages) & 1, abort));
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars.v_full[j % kVS], (j / kVS) & 1, abort));
         if (!ok) break;
         if (tid >= nk) {
-          uint8_t* sv = gbase + kSmemKV + (j % kStages) * 2 * kTileBytes + kTileBytes;
+          uint8_t* sv = gbase + kSmemV + (j % kVS) * kTileBytes;
           const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -579,156 +672,101 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
             *reinterpret_cast<uint4*>(sv + kHalfBytes + tid * 128 + c * 16) = z;
           }
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
-      uint8_t* prow = gbase + kSmemP + tid * 128;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint4 v;
-        v.x = pack_bf16(s[8 * c + 0], s[8 * c + 1]);
-        v.y = pack_bf16(s[8 * c + 2], s[8 * c + 3]);
-        v.z = pack_bf16(s[8 * c + 4], s[8 * c + 5]);
-        v.w = pack_bf16(s[8 * c + 6], s[8 * c + 7]);
-        const int half = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4*>(prow + half * kHalfBytes + ((cc ^ (tid & 7)) << 4)) = v;
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.p_full);
+      if (lane == 0) mbar_arrive(&bars.p_full[j & 1]);
     }
-    // epilogue
+    // ------------------------------------------------------------ epilogue
     if (ok && ntot > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (ntot - 1) & 1, abort));
-    if (ok) {
-      fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
-      if (p.nchunk == 1) {
-        // single chunk: this CTA holds the whole result
-        const bool good = my_ok && !bad_len;
-        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + row_node * p.o_st + row_head * p.o_sh;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(trow + kColO + c * 32, v);
-          tmem_wait_ld();
-          if (row_valid) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint4 w;
-              if (good) {
-                w.x = pack_bf16(v[e] * inv, v[e + 1] * inv);
-                w.y = pack_bf16(v[e + 2] * inv, v[e + 3] * inv);
-                w.z = pack_bf16(v[e + 4] * inv, v[e + 5] * inv);
-                w.w = pack_bf16(v[e + 6] * inv, v[e + 7] * inv);
-              } else {
-                w.x = w.y = w.z = w.w = pack_bf16(NAN, NAN);
-              }
-              *reinterpret_cast<uint4*>(o + c * 32 + e) = w;
-            }
-          }
-        }
-        if (row_valid) {
-          if (p.lse) p.lse[(static_cast<int64_t>(b) * p.T + row_node) * p.Hq + row_head] = good ? lse : NAN;
-          if (!my_ok) set_status(p.status, TV_DEV_BAD_PARENT);
-          if (bad_len && row_node == 0 && row_head == 0) set_status(p.status, TV_DEV_BAD_LEN);
-        }
-      } else {
-        float* po = row_valid ? p.part_o + part_row(p, chunk, b, row_node, row_head) * kD : nullptr;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(trow + kColO + c * 32, v);
-          tmem_wait_ld();
-          if (row_valid) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4*>(po + c * 32 + e) =
-                  (l_run > 0.f) ? make_float4(v[e] * inv, v[e + 1] * inv, v[e + 2] * inv, v[e + 3] * inv)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-        if (row_valid) {
-          // invalid rows carry NaN into the merge
-          const bool good = my_ok && !bad_len;
-          p.part_lse[part_row(p, chunk, b, row_node, row_head)] = good ? lse : NAN;
-          if (has_tree && !my_ok) set_status(p.status, TV_DEV_BAD_PARENT);
-          if (bad_len && chunk == 0 && row_node == 0 && row_head == 0) set_status(p.status, TV_DEV_BAD_LEN);
-        }
-      }
-    }
-  }
-  // ------------------------------------------------------------------ teardown
-  fence_before();
-  __syncthreads();
-  if (*abort) {
-    if (tid == 0) set_status(p.status, TV_DEV_TIMEOUT);
-    if (row_valid) {
-      if (p.nchunk == 1) {
-        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + row_node * p.o_st + row_head * p.o_sh;
-        for (int c = 0; c < kD; ++c) o[c] = __float2bfloat16(NAN);
-      } else {
-        p.part_lse[part_row(p, chunk, b, row_node, row_head)] = NAN;
-      }
-    }
-  }
-  if (warp == 5) {
     fence_after();
+    const bool have = ok && l_run > 0.f;
+    const float inv = have ? 1.f / l_run : 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      tmem_ld32(trow + kColO + c * 32, orow + c * 32);
+      tmem_wait_ld();
+    }
+#pragma unroll
+    for (int e = 0; e < kD; ++e) orow[e] = have ? orow[e] * inv : 0.f;
+    const bool good = !(has_tree && !my_ok) && !bad_len && ok;
+    my_lse2 = !good ? NAN : (l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY);
+    if (row_valid && has_tree && !my_ok) set_status(p.status, TV_DEV_BAD_PARENT);
+    if (bad_len && has_tree && tid == 0) set_status(p.status, TV_DEV_BAD_LEN);
+  }
+
+  // ------------------------------------------------------------ cluster merge
+  // Row t of the tile is merged by CTA t / per.  Every CTA pushes its rows
+  // (normalised O, fp32) and their log2-sum-exp into the owners' shared
+  // memory (the K rings, idle once all CTAs have left their main loops);
+  // each owner then merges its rows from local shared memory.
+  const int rows_here = nodes_here * G;
+  const int per = (rows_here + C - 1) / C;
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  fence_before();
+  cl.sync();                  // every CTA is past its main loop
+  fence_after();
+  if (warp == kWarpMma) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
-}
-
-// Log-sum-exp merge of the chunk partials of the tensor-core kernel: one
-// warp per (sequence, node, query head); lane c holds chunk c's lse, lane l
-// accumulates dimensions 4l .. 4l+3 with every chunk's load in flight.  The
-// partials of rows that are invalid (malformed parent chain, prefix length
-// out of range) carry lse = NaN and the merged row is NaN.
-__global__ void __launch_bounds__(256) attn_tc_merge_kernel(AttnParams p) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= static_cast<int64_t>(p.B) * p.T * p.Hq) return;
-  const int h = static_cast<int>(row % p.Hq);
-  const int i = static_cast<int>((row / p.Hq) % p.T);
-  const int b = static_cast<int>(row / (static_cast<int64_t>(p.Hq) * p.T));
-  const int n = p.n_nodes ? p.n_nodes[b] : p.T;
-  if (n < 0 || n > p.T || i >= n) return;
-  // a NaN partial lse marks a row the tensor-core kernel found invalid
-  const int np = p.nchunk;
-  float lc = -INFINITY;
-  if (lane < np) lc = __ldcg(&p.part_lse[part_row(p, lane, b, i, h)]);
-  const bool good = !__any_sync(0xffffffffu, lc != lc);
-  if (!good) lc = -INFINITY;
-  const float M = warp_max(lc);
-  const float wl = (lane < np && lc > -INFINITY) ? __expf(lc - M) : 0.f;
-  const float den = warp_sumf(wl);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c0 = 0; c0 < np; c0 += 8) {
-    float4 v[8];
+  if (tid < rows_here) {
+    const int owner = tid / per, r = chunk * per + (tid - owner * per);
+    float* dst = cl.map_shared_rank(reinterpret_cast<float*>(gbase + kSmemInbox), owner) + r * kD;
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      v[u] = (c0 + u < np) ? __ldcg(reinterpret_cast<const float4*>(p.part_o + part_row(p, c0 + u, b, i, h) * kD) + lane)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float w = __shfl_sync(0xffffffffu, wl, (c0 + u) & 31);
-      if (c0 + u < np) {
-        acc.x = fmaf(w, v[u].x, acc.x); acc.y = fmaf(w, v[u].y, acc.y);
-        acc.z = fmaf(w, v[u].z, acc.z); acc.w = fmaf(w, v[u].w, acc.w);
+    for (int q = 0; q < kD / 4; ++q)
+      *reinterpret_cast<float4*>(dst + ((q ^ (r & 7)) * 4)) =
+          make_float4(orow[4 * q], orow[4 * q + 1], orow[4 * q + 2], orow[4 * q + 3]);
+    cl.map_shared_rank(&bars, owner)->in_lse[r] = my_lse2;
+  }
+  if (tid < C) cl.map_shared_rank(&bars, tid)->in_abort[chunk] = *abort;
+  if (*abort && tid == 0) set_status(p.status, TV_DEV_TIMEOUT);
+  cl.sync();                  // the pushes have landed
+  {
+    const float* inbox = reinterpret_cast<const float*>(gbase + kSmemInbox);
+    const int r0 = chunk * per;
+    for (int lt = warp; lt < per && r0 + lt < rows_here; lt += kThreads / 32) {
+      const int t = r0 + lt;
+      float lc = -INFINITY;
+      int ab = 0;
+      if (lane < C) {
+        lc = bars.in_lse[lane * per + lt];
+        ab = bars.in_abort[lane];
       }
+      const bool bad = __any_sync(0xffffffffu, (lc != lc) || ab != 0);
+      if (lc != lc) lc = -INFINITY;
+      const float M = warp_max(lc);
+      const float wl = (lc > -INFINITY) ? ex2_approx(lc - M) : 0.f;
+      const float den = warp_sumf(wl);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < kMaxCluster; ++c) {
+        const float w = __shfl_sync(0xffffffffu, wl, c);
+        if (c < C && w != 0.f) {
+          const int r = c * per + lt;
+          const float4 v = *reinterpret_cast<const float4*>(inbox + r * kD + ((lane ^ (r & 7)) * 4));
+          acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+          acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+        }
+      }
+      const bool okr = !bad && den > 0.f;
+      const float iv = okr ? 1.f / den : 0.f;
+      uint2 wv;
+      if (okr) {
+        wv.x = pack_bf16(acc.x * iv, acc.y * iv);
+        wv.y = pack_bf16(acc.z * iv, acc.w * iv);
+      } else {
+        wv.x = wv.y = pack_bf16(NAN, NAN);
+      }
+      const int node = i0 + t / G, head = g * G + t % G;
+      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + node * p.o_st + head * p.o_sh;
+      *reinterpret_cast<uint2*>(o + lane * 4) = wv;
+      if (lane == 0 && p.lse)
+        p.lse[(static_cast<int64_t>(b) * p.T + node) * p.Hq + head] =
+            okr ? (M + __log2f(den)) * 0.6931471805599453f : NAN;
     }
   }
-  const bool ok = good && den > 0.f;
-  const float inv = ok ? 1.f / den : 0.f;
-  uint2 wv;
-  if (ok) {
-    wv.x = pack_bf16(acc.x * inv, acc.y * inv);
-    wv.y = pack_bf16(acc.z * inv, acc.w * inv);
-  } else {
-    wv.x = wv.y = pack_bf16(NAN, NAN);
-  }
-  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + i * p.o_st + h * p.o_sh;
-  *reinterpret_cast<uint2*>(o + lane * 4) = wv;
-  if (lane == 0 && p.lse) p.lse[row] = ok ? M + __logf(den) : NAN;
 }
 
 // ------------------------------------------------------------------ host side
@@ -797,9 +835,41 @@ bool attn_tc_supported(const tv_attn_args* a) {
   return major == 10 && minor == 0;
 }
 
+int attn_tc_active_clusters(int c) {
+  // clusters of c chunk CTAs that can be resident at once (cached per device)
+  static int cached[64][kMaxCluster + 1];
+  static bool done[64][kMaxCluster + 1];
+  int dev = 0;
+  if (c < 1 || c > kMaxCluster) return 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (done[dev][c]) return cached[dev][c];
+  int n = 0;
+  const size_t smem = kSmemBytes + 1024;
+  if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(c, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  cached[dev][c] = n;
+  done[dev][c] = true;
+  return n;
+}
+
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   const int G = p.G;
+  if (p.nchunk < 1 || p.nchunk > kMaxCluster) return cudaErrorInvalidValue;
   if (!make_map(&mq, p.q, p.d, p.Hq, p.T, p.B, p.q_sh, p.q_st, p.q_sb, G, kRows / G) ||
       !make_map(&mk, p.kc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, kKeys) ||
       !make_map(&mv, p.vc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, kKeys))
@@ -809,12 +879,20 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream) {
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int ntiles = (p.T + p.node_tile - 1) / p.node_tile;
-  dim3 grid(p.nchunk, ntiles, p.B * p.Hkv);
-  attn_tc_kernel<<<grid, kThreads, smem, stream>>>(mq, mk, mv, p);
-  if (p.nchunk > 1) {
-    const int64_t rows = static_cast<int64_t>(p.B) * p.T * p.Hq;
-    attn_tc_merge_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
-  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.nchunk, ntiles, p.B * p.Hkv);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.nchunk;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, mq, mk, mv, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

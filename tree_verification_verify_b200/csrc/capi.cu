@@ -15,6 +15,7 @@ cudaError_t launch_expand_init(const tv_expand_args* a, int root_token, cudaStre
 cudaError_t launch_expand(const tv_expand_args* a, cudaStream_t stream);
 bool attn_tc_supported(const tv_attn_args* a);
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream);
+int attn_tc_active_clusters(int c);
 cudaError_t launch_block_means(const AttnParams& p, float* kbar, cudaStream_t stream);
 cudaError_t launch_block_select(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attn_sparse(const AttnParams& p, cudaStream_t stream);
@@ -75,33 +76,48 @@ AttnPlan plan_attn(const tv_attn_args* a) {
     pl.nchunk = pl.sparse ? 1 : 0;
     pl.chunk_len = 128;
   } else {
-    // about four waves of CTAs (balance across ragged prefixes), but at least four 128-key tiles per
-    // chunk for the tensor-core kernel (its pipeline and the partial
-    // write-back are amortised over the chunk), and at most 31 chunks so
-    // that the merge reads every partial of a row with one warp
+    // about four waves of CTAs (balance across ragged prefixes); the
+    // tensor-core kernel takes at least four 128-key tiles per chunk (its
+    // pipeline is amortised over the chunk) and at most one cluster of
+    // chunks per row tile (it merges them over distributed shared memory);
+    // the CUDA-core path takes at most 31 chunks so that its merge reads
+    // every partial of a row with one warp
     const int64_t target = 4LL * num_sms();
     int64_t want = (target + units - 1) / units;
     int64_t maxc = (a->Lmax + 127) / 128;
-    if (pl.tc) maxc = (a->Lmax + 511) / 512;
     if (maxc > 31) maxc = 31;
     if (want < 1) want = 1;
     if (want > maxc) want = maxc;
     int64_t len = (a->Lmax + want - 1) / want;
     len = (len + 127) / 128 * 128;
+    if (pl.tc) {
+      // tensor-core kernel: c chunks of a row tile form one cluster.  Cost
+      // model in tile times: each CTA pays about three tiles of latency
+      // (start-up, first loads, merge) plus its chunk's tiles, and the row
+      // tiles' clusters run in waves of what the device holds at once.
+      const int64_t tiles = (a->Lmax + 127) / 128;
+      double best = 1e300;
+      int64_t best_len = tiles;
+      for (int c = 1; c <= 8; ++c) {
+        const int64_t lt = (tiles + c - 1) / c;
+        if (c > 1 && lt < 4) break;                       // at least four tiles per chunk
+        if ((tiles + lt - 1) / lt != c) continue;          // c chunks not realisable
+        const int act = attn_tc_active_clusters(c);
+        if (act <= 0) continue;
+        const double waves = static_cast<double>((units + act - 1) / act);
+        const double cost = waves * (3.0 + static_cast<double>(lt));
+        if (cost < best) { best = cost; best_len = lt; }
+      }
+      len = best_len * 128;
+    }
     pl.chunk_len = static_cast<int>(len);
     pl.nchunk = static_cast<int>((a->Lmax + len - 1) / len);
   }
-  if (pl.tc) {
-    // the merge uses one ticket per (sequence, kv head, row tile) group
-    const int64_t groups = static_cast<int64_t>(a->B) * a->Hkv * ntiles;
-    if (groups > kMaxTickets) { pl.nchunk = (a->Lmax > 0) ? 1 : 0; pl.chunk_len = a->Lmax > 0 ? ((a->Lmax + 127) / 128) * 128 : 128; }
-    if (pl.nchunk == 0) { pl.nchunk = 1; pl.chunk_len = 128; }
-  }
+  if (pl.tc && pl.nchunk == 0) { pl.nchunk = 1; pl.chunk_len = 128; }
   const size_t rows = static_cast<size_t>(a->B) * a->T * a->Hq;
-  // the tensor-core path keeps a single chunk's result on chip; the other
-  // paths always merge (prefix chunks + the tree-path partial)
-  const size_t nparts = pl.tc ? (pl.nchunk > 1 ? static_cast<size_t>(pl.nchunk) : 0)
-                              : static_cast<size_t>(pl.nchunk) + 1;
+  // the tensor-core path merges its chunks on chip; the other paths merge
+  // partials (prefix chunks + the tree-path partial) through the workspace
+  const size_t nparts = pl.tc ? 0 : static_cast<size_t>(pl.nchunk) + 1;
   size_t off = kTicketBytes;
   pl.off_o = off;  off = align256(off + nparts * rows * a->d * sizeof(float));
   pl.off_lse = off; off = align256(off + nparts * rows * sizeof(float));
@@ -138,7 +154,7 @@ extern "C" int32_t tv_attn_launches(const tv_attn_args* a) {
   if (a->B == 0 || a->T == 0) return 0;
   const AttnPlan pl = plan_attn(a);
   if (pl.sparse) return (a->k_block_mean ? 0 : 1) + 4;
-  if (pl.tc) return pl.nchunk > 1 ? 2 : 1;
+  if (pl.tc) return 1;
   return 3;
 }
 
@@ -185,7 +201,7 @@ extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws
     if (e != cudaSuccess) return from_cuda(e);
     e = launch_attn_sparse(p, s);
   } else if (pl.tc) {
-    // one kernel: prefix tiles, tree tiles and the split merge
+    // one kernel: prefix tiles, tree tiles and the cluster merge of the chunks
     return from_cuda(launch_attn_tc(p, s));
   } else {
     e = launch_attn_simt(p, s);
