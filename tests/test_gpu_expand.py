@@ -147,3 +147,29 @@ def test_specexec70b_full_build():
     assert compared >= 8
     if not near:
         assert compared == ec.n_calls() == 16
+
+
+def test_crowded_boundary_bin_ties():
+    """Exact ties at the top of the rows: 10% of a 50000-token vocabulary
+    share the maximal logit, so the selection boundary falls inside a run of
+    identical values (the crowded-bin path); the order inside the run is
+    the token index on both sides.  Exact ties make the oracle's rank gaps
+    zero, so the rounds are compared directly."""
+    import tree_verification_verify_b200 as tv
+    V, Bsel, budget = 50000, 64, 512
+    g = torch.Generator().manual_seed(11)
+    st = tv.tree_expand_init(budget, V, Bsel)
+    os_ = OState(budget, 0)
+    frontier = [0]
+    for call in range(3):
+        z = (torch.rand(len(frontier), V, generator=g) < 0.1).float() * 2.0 - 1.0
+        rows = torch.tensor(frontier, dtype=torch.int32, device="cuda")
+        tv.tree_expand_topb(st, z.cuda(), rows)
+        new = expand_call(os_, z, frontier, Bsel)
+        torch.cuda.synchronize()
+        n = os_.n_nodes
+        np.testing.assert_array_equal(st.parent.cpu().numpy()[:n], np.array(os_.parent))
+        np.testing.assert_array_equal(st.token.cpu().numpy()[:n], np.array(os_.token))
+        np.testing.assert_allclose(st.logp.cpu().numpy()[:n], np.array(os_.logp), rtol=0, atol=1e-12)
+        assert st.frontier.cpu().numpy()[:len(new)].tolist() == new
+        frontier = new

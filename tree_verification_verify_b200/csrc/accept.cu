@@ -15,16 +15,19 @@
 //
 // Layout of a row pass.  A thread-block cluster of C CTAs (C <= 8) owns one
 // node row; CTA rank r owns a contiguous slice of 512-element segments.  A
-// warp owns a segment at a time: four warp-wide 16-byte loads, lane l holding
-// elements 128k + 4l .. 128k + 4l + 3 (k = 0..3); full segments are read
-// without bounds checks.  Cross-CTA sums and maxima go
+// warp owns a segment at a time, lane l holding elements 128k + 4l ..
+// 128k + 4l + 3 (k = 0..3).  Aligned rows are streamed by bulk copies: each
+// warp keeps three segments (z and q) in flight in its own shared-memory
+// ring; other rows are read with plain loads.  Cross-CTA sums and maxima go
 // through distributed shared memory (double-buffered slots, one cluster
 // barrier per reduction); every CTA computes the same reduced values and so
 // takes the same branches.
 //
-// Arithmetic.  The row maximum M is found first; every element weight is
-// then e_t = 2^(z_t * k - M * k) with k = log2(e) / tau (one FFMA and one
-// ex2.approx), the unnormalised softmax.  Residuals are parametrised as
+// Arithmetic.  Every element weight is e_t = 2^(z_t * k - M * k) with
+// k = log2(e) / tau and M the row maximum (one FFMA and one ex2.approx), the
+// unnormalised softmax.  The first pass keeps, per segment, the maximum m_s
+// and the sum of 2^((z - m_s) k); once the per-CTA maxima are gathered, the
+// row sum and the segment sums are brought to the frame of M.  Residuals are parametrised as
 // r = (p - c q)^+ / D with p = e / s: rejecting a child with the current
 // (c, D) gives c' = c + D and D' = sum_t (p_t - c' q_t)^+, one pass.
 // Weights are fp32; each lane's four weights are summed in fp32, segment
@@ -76,6 +79,11 @@ constexpr int kAcceptWarps = kAcceptThreads / kWarp;
 constexpr int kSeg = 512;               // elements per segment
 constexpr int kSub = 128;               // elements of one warp-wide float4 load
 constexpr int kMaxSegPerCta = 128;      // 65536 elements per CTA
+constexpr int kRing = 3;                // segments in flight per warp (bulk copies)
+constexpr uint32_t kSegBytes = kSeg * 4;
+constexpr uint32_t kStageBytes = 2 * kSegBytes;               // z then q
+constexpr size_t kRingBytes = static_cast<size_t>(kAcceptWarps) * kRing * kStageBytes;   // 96 KB
+constexpr uint32_t kRingWait = 1u << 22;
 
 // ------------------------------------------------------------ shared state
 
@@ -91,13 +99,22 @@ struct AcceptShared {
   int red_i[kAcceptWarps];
   int wofs[kAcceptWarps];
   int clist[kAcceptThreads];
+  int ctok[kAcceptThreads];     // first window of children: tokens, z and q at them
+  float cz[kAcceptThreads];
+  float cq[kAcceptThreads];
   int bc_int[4];
   double bc_dbl[4];
   Slot slot[2];
+  double cu[kAcceptThreads];    // first window of children: their uniforms
   double rank_tot[8];           // per-CTA totals of the current weights
   float seg_a[kMaxSegPerCta];   // segment sums of the current weights
-  float seg_b[kMaxSegPerCta];   // scratch for a residual pass
+  float seg_b[kMaxSegPerCta];   // scratch for a residual pass (first pass: segment maxima)
+  uint64_t ring_bar[kAcceptWarps * kRing];
 };
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -185,32 +202,157 @@ __device__ __forceinline__ void load_seg(const float* __restrict__ row, int s0, 
   }
 }
 
+// ---------------------------------------------------------- segment streams
+// A warp visits its segments s = warp, warp + 8, ... of the CTA's slice in
+// order.  When the rows allow it (16-byte aligned rows, V a multiple of 4)
+// lane 0 keeps kRing segments in flight with bulk copies into the warp's
+// ring in shared memory (one mbarrier per ring stage); otherwise the lanes
+// load each segment directly.  The same slice is streamed once per pass.
+
+__device__ __forceinline__ void ring_expect(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void ring_copy(uint32_t dst, const float* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Bounded wait on phase `parity` of a ring barrier; false when it expired.
+__device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_addr(bar);
+  for (uint32_t it = 0; it < kRingWait; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+struct SegStream {
+  const float* zr;
+  const float* qr;
+  bool zvec, qvec;      // 16-byte aligned rows (plain loads)
+  bool readq;           // stream q as well
+  bool bulk;            // bulk copies into the ring
+  int V, seg0, nloc;
+  uint32_t ring;        // shared address of this warp's ring
+  uint64_t* bar;        // this warp's kRing barriers
+  uint32_t count;       // segments this warp has streamed (all passes)
+  bool dead;            // a ring wait expired: the stream delivers fill values
+};
+
+__device__ __forceinline__ void seg_issue(const SegStream& st, int sl, uint32_t stage) {
+  const int s0 = (st.seg0 + sl) * kSeg;
+  const uint32_t bytes = static_cast<uint32_t>(min(kSeg, st.V - s0)) * 4u;
+  uint64_t* bar = st.bar + stage;
+  ring_expect(bar, st.readq ? 2u * bytes : bytes);
+  ring_copy(st.ring + stage * kStageBytes, st.zr + s0, bytes, bar);
+  if (st.readq) ring_copy(st.ring + stage * kStageBytes + kSegBytes, st.qr + s0, bytes, bar);
+}
+
+// One pass over the warp's segments: f(sl, s0, z[4], q[4]) per segment
+// (sl the segment's index in the slice, s0 its first element; the lane
+// holds elements s0 + 128k + 4l ..; past the row end z reads zfill and q 0).
+template <class F>
+__device__ __forceinline__ void stream_pass(SegStream& st, float zfill, F&& f) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ns = warp < st.nloc ? (st.nloc - warp + kAcceptWarps - 1) / kAcceptWarps : 0;
+  if (!st.bulk) {
+    for (int i = 0; i < ns; ++i) {
+      const int sl = warp + i * kAcceptWarps;
+      const int s0 = (st.seg0 + sl) * kSeg;
+      float4 zv[4], qv[4];
+      load_seg(st.zr, s0, st.V, st.zvec, zfill, zv);
+      if (st.readq) load_seg(st.qr, s0, st.V, st.qvec, 0.f, qv);
+      else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) qv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      f(sl, s0, zv, qv);
+    }
+    return;
+  }
+  const uint32_t c0 = st.count;
+  if (lane == 0 && !st.dead)
+    for (int i = 0; i < min(kRing, ns); ++i) seg_issue(st, warp + i * kAcceptWarps, (c0 + i) % kRing);
+  for (int i = 0; i < ns; ++i) {
+    const uint32_t g = c0 + i, stage = g % kRing;
+    const int sl = warp + i * kAcceptWarps;
+    const int s0 = (st.seg0 + sl) * kSeg;
+    if (!st.dead && !__all_sync(0xffffffffu, ring_wait(st.bar + stage, (g / kRing) & 1))) {
+      // expired: issue nothing more, let the copies in flight land (bounded)
+      st.dead = true;
+      if (lane == 0)
+        for (int j = i; j < min(i + kRing, ns); ++j) ring_wait(st.bar + (c0 + j) % kRing, ((c0 + j) / kRing) & 1);
+      __syncwarp();
+    }
+    float4 zv[4], qv[4];
+    if (!st.dead) {
+      const uint8_t* stg = reinterpret_cast<const uint8_t*>(__cvta_shared_to_generic(st.ring + stage * kStageBytes));
+      const float4* z4 = reinterpret_cast<const float4*>(stg) + lane;
+      const float4* q4 = reinterpret_cast<const float4*>(stg + kSegBytes) + lane;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        zv[k] = z4[32 * k];
+        qv[k] = st.readq ? q4[32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      if (s0 + kSeg > st.V) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e0 = s0 + k * kSub + 4 * lane;
+          if (e0 + 0 >= st.V) { zv[k].x = zfill; qv[k].x = 0.f; }
+          if (e0 + 1 >= st.V) { zv[k].y = zfill; qv[k].y = 0.f; }
+          if (e0 + 2 >= st.V) { zv[k].z = zfill; qv[k].z = 0.f; }
+          if (e0 + 3 >= st.V) { zv[k].w = zfill; qv[k].w = 0.f; }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        zv[k] = make_float4(zfill, zfill, zfill, zfill);
+        qv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    f(sl, s0, zv, qv);
+    __syncwarp();
+    if (!st.dead && i + kRing < ns && lane == 0) {
+      // the lanes' reads of this stage are done before the copy overwrites it
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      seg_issue(st, warp + (i + kRing) * kAcceptWarps, stage);
+    }
+  }
+  st.count = c0 + ns;
+}
+
 // One pass over this CTA's slice: segment sums of the current weights into
 // seg_out; returns the slice total (fp64).  Past the row end the logits read
 // -FLT_MAX, whose weight is 0.
-template <bool READQ>
-__device__ double weight_pass(const float* zr, const float* qr, bool zvec, bool qvec, int V, int seg0, int nloc,
-                              const Frame& f, float* seg_out, AcceptShared& sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ double weight_pass(SegStream& st, const Frame& f, float* seg_out, AcceptShared& sh) {
+  const int lane = threadIdx.x & 31;
   double tot = 0.0;
-  for (int s = warp; s < nloc; s += kAcceptWarps) {
-    const int s0 = (seg0 + s) * kSeg;
-    float4 zv[4], qv[4];
-    load_seg(zr, s0, V, zvec, -FLT_MAX, zv);
-    if (READQ) load_seg(qr, s0, V, qvec, 0.f, qv);
+  stream_pass(st, -FLT_MAX, [&](int sl, int, const float4 (&zv)[4], const float4 (&qv)[4]) {
     float g = 0.f;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const float4 q4 = READQ ? qv[k] : make_float4(0.f, 0.f, 0.f, 0.f);
-      g += weight(zv[k].x, q4.x, f.k, f.zoff, f.inv_s, f.c, f.resid);
-      g += weight(zv[k].y, q4.y, f.k, f.zoff, f.inv_s, f.c, f.resid);
-      g += weight(zv[k].z, q4.z, f.k, f.zoff, f.inv_s, f.c, f.resid);
-      g += weight(zv[k].w, q4.w, f.k, f.zoff, f.inv_s, f.c, f.resid);
+      g += weight(zv[k].x, qv[k].x, f.k, f.zoff, f.inv_s, f.c, f.resid);
+      g += weight(zv[k].y, qv[k].y, f.k, f.zoff, f.inv_s, f.c, f.resid);
+      g += weight(zv[k].z, qv[k].z, f.k, f.zoff, f.inv_s, f.c, f.resid);
+      g += weight(zv[k].w, qv[k].w, f.k, f.zoff, f.inv_s, f.c, f.resid);
     }
     const float ss = warp_sum_f(g);
-    if (lane == 0) seg_out[s] = ss;
+    if (lane == 0) seg_out[sl] = ss;
     tot += static_cast<double>(ss);
-  }
+  });
   return block_sum_d(lane == 0 ? tot : 0.0, sh);
 }
 
@@ -319,13 +461,28 @@ __device__ void slice_search(const float* zr, const float* qr, bool zvec, bool q
 // ------------------------------------------------------------ the walk
 
 // Called by every thread of one CTA: thread 0 follows the accepted children
-// from the root, then the block pads the outputs with -1.
-__device__ void accept_walk(const AcceptParams& p, int b, int n, AcceptShared& sh) {
+// from the root, then the block pads the outputs with -1.  When they fit,
+// the sequence's decisions are first copied to `scratch` (shared memory) by
+// the whole block, so that the walk's dependent reads stay on chip.
+__device__ void accept_walk(const AcceptParams& p, int b, int n, AcceptShared& sh, AcceptDec* scratch,
+                            int scratch_cap) {
   const int T = p.T;
   int32_t* acc = p.acc_nodes + static_cast<int64_t>(b) * T;
   int32_t* out = p.out_tokens + static_cast<int64_t>(b) * (T + 1);
   const int32_t* tok = p.tok + b * p.tok_sb;
   const bool walk = (n > 0 && n <= T);
+  const AcceptDec* dsrc = p.dec + static_cast<int64_t>(b) * T;
+  const bool local = walk && n <= scratch_cap;
+  if (local) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      AcceptDec d;
+      d.child = __ldcg(&dsrc[i].child);
+      d.token = __ldcg(&dsrc[i].token);
+      d.margin = __ldcg(&dsrc[i].margin);
+      scratch[i] = d;
+    }
+    __syncthreads();
+  }
   if (threadIdx.x == 0) {
     int len = 0;
     double mg = INFINITY;
@@ -333,10 +490,17 @@ __device__ void accept_walk(const AcceptParams& p, int b, int n, AcceptShared& s
       int c = 0;
       int bonus = -1;
       for (int step = 0; step < n; ++step) {
-        const AcceptDec* dp = p.dec + static_cast<int64_t>(b) * T + c;
-        const int child = __ldcg(&dp->child);
-        const int token = __ldcg(&dp->token);
-        mg = fmin(mg, __ldcg(&dp->margin));
+        int child, token;
+        if (local) {
+          child = scratch[c].child;
+          token = scratch[c].token;
+          mg = fmin(mg, scratch[c].margin);
+        } else {
+          const AcceptDec* dp = dsrc + c;
+          child = __ldcg(&dp->child);
+          token = __ldcg(&dp->token);
+          mg = fmin(mg, __ldcg(&dp->margin));
+        }
         if (child >= 0 && child < n) {
           acc[len] = child;
           out[len] = tok[child];
@@ -365,9 +529,10 @@ __device__ void accept_walk(const AcceptParams& p, int b, int n, AcceptShared& s
 
 // ------------------------------------------------------------ node kernel
 
-__global__ void __launch_bounds__(kAcceptThreads, 3)
+__global__ void __launch_bounds__(kAcceptThreads, 2)
 accept_node_kernel(AcceptParams p) {
   __shared__ AcceptShared sh;
+  extern __shared__ __align__(128) uint8_t ring_smem[];
   cg::cluster_group cl = cg::this_cluster();
   const int C = p.C;
   const int rank = static_cast<int>(cl.block_rank());
@@ -378,7 +543,7 @@ accept_node_kernel(AcceptParams p) {
     // nothing to decide: the first CTA writes the empty result
     if (c == 0 && rank == 0) {
       if (n != 0 && tid == 0) set_status(p.status, TV_DEV_BAD_LEN);
-      accept_walk(p, b, n, sh);
+      accept_walk(p, b, n, sh, nullptr, 0);
     }
     return;                                  // the whole cluster leaves together
   }
@@ -408,27 +573,67 @@ accept_node_kernel(AcceptParams p) {
   const bool greedy = (p.mode == TV_ACCEPT_GREEDY);
   const bool specsample = (p.mode == TV_ACCEPT_SPECSAMPLE);
   int has_child = 0;
+  int cnt0 = 0;                 // children in the first window [c + 1, c + 1 + blockDim)
   if (specsample) {
-    int fl = 0;
-    for (int j = c + 1 + tid; j < n && !fl; j += blockDim.x) fl = (par[j] == c);
+    // the first window of children, in node order, and whether more follow
+    const int j = c + 1 + tid;
+    const bool is = (j < n) && par[j] == c;
+    const unsigned m = __ballot_sync(0xffffffffu, is);
+    if (lane == 0) sh.red_i[warp] = __popc(m);
+    __syncthreads();
+    if (tid == 0) {
+      int acc = 0;
+      for (int w = 0; w < kAcceptWarps; ++w) { sh.wofs[w] = acc; acc += sh.red_i[w]; }
+      sh.bc_int[3] = acc;
+    }
+    __syncthreads();
+    if (is) sh.clist[sh.wofs[warp] + __popc(m & ((1u << lane) - 1u))] = j;
+    cnt0 = sh.bc_int[3];
+    int fl = cnt0 > 0;
+    for (int jj = c + 1 + static_cast<int>(blockDim.x) + tid; jj < n && !fl; jj += blockDim.x) fl = (par[jj] == c);
     has_child = __syncthreads_or(fl);
   }
   const bool read_q = specsample && has_child;
   const float* qr = read_q ? p.q + b * p.q_sb + c * p.q_st : nullptr;
   const bool qvec = read_q && ((reinterpret_cast<uintptr_t>(qr) & 15u) == 0);
+  if (read_q && tid < cnt0) {
+    // the first window's point values, loaded while the first pass streams
+    const int x = tok[sh.clist[tid]];
+    const bool okx = x >= 0 && x < V;
+    sh.ctok[tid] = x;
+    sh.cz[tid] = okx ? zr[x] : 0.f;
+    sh.cq[tid] = okx ? qr[x] : 0.f;
+    sh.cu[tid] = accept_uniform(p.seed, p.step, b, c, tid, kTagChild);
+  }
+  if (!greedy && tid == kAcceptThreads - 1)
+    sh.bc_dbl[3] = accept_uniform(p.seed, p.step, b, c, 0, specsample ? kTagResidual : kTagSpecExec);
 
-  // ---- pass A: the row maximum (greedy: its first index), finiteness
-  float bv = -INFINITY;
-  int bi = INT_MAX;
-  bool bad = false;
-  float nf = 0.f;                 // x * 0 turns any non-finite x into NaN
-  float qmin = 0.f;
-  for (int s = warp; s < nloc; s += kAcceptWarps) {
-    const int s0 = (seg0 + s) * kSeg;
-    float4 v[4], qv[4];
-    load_seg(zr, s0, V, zvec, greedy ? -INFINITY : -FLT_MAX, v);
-    if (read_q) load_seg(qr, s0, V, qvec, 0.f, qv);
-    if (greedy) {
+  SegStream st;
+  st.zr = zr; st.qr = qr; st.zvec = zvec; st.qvec = qvec; st.readq = read_q;
+  st.bulk = zvec && (V % 4 == 0) && (!read_q || qvec);
+  st.V = V; st.seg0 = seg0; st.nloc = nloc;
+  st.ring = smem_addr(ring_smem) + warp * kRing * kStageBytes;
+  st.bar = sh.ring_bar + warp * kRing;
+  st.count = 0;
+  st.dead = false;
+  if (st.bulk) {
+    if (lane == 0) {
+      for (int r = 0; r < kRing; ++r)
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(st.bar + r)) : "memory");
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+  }
+
+  float M = -INFINITY;
+  int gbad = 0;
+  double ssum = 0.0;
+  if (greedy) {
+    // ---- the row maximum and its first index; NaN makes the row non-finite
+    float bv = -INFINITY;
+    int bi = INT_MAX;
+    bool bad = false;
+    stream_pass(st, -INFINITY, [&](int, int s0, const float4 (&v)[4], const float4 (&)[4]) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int e0 = s0 + k * kSub + lane * 4;
@@ -442,75 +647,113 @@ accept_node_kernel(AcceptParams p) {
           }
         }
       }
-    } else {
+    });
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        bv = fmaxf(fmaxf(bv, v[k].x), fmaxf(v[k].y, fmaxf(v[k].z, v[k].w)));
-        nf = fmaf(v[k].x, 0.f, nf); nf = fmaf(v[k].y, 0.f, nf);
-        nf = fmaf(v[k].z, 0.f, nf); nf = fmaf(v[k].w, 0.f, nf);
-        if (read_q) {
-          qmin = fminf(qmin, fminf(fminf(qv[k].x, qv[k].y), fminf(qv[k].z, qv[k].w)));
-          nf = fmaf(qv[k].x, 0.f, nf); nf = fmaf(qv[k].y, 0.f, nf);
-          nf = fmaf(qv[k].z, 0.f, nf); nf = fmaf(qv[k].w, 0.f, nf);
-        }
-      }
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
-  }
-  if (!greedy && (nf != nf || qmin < 0.f)) bad = true;
-  if (!greedy) bi = 0;
+    const int any_bad = __syncthreads_or(bad ? 1 : 0);
+    if (lane == 0) { sh.red_f[warp] = bv; sh.red_i[warp] = bi; }
+    __syncthreads();
+    {
+      float v = -INFINITY;
+      int i = INT_MAX;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-  }
-  const int any_bad = __syncthreads_or(bad ? 1 : 0);
-  if (lane == 0) { sh.red_f[warp] = bv; sh.red_i[warp] = bi; }
-  __syncthreads();
-  {
-    float v = -INFINITY;
-    int i = INT_MAX;
-#pragma unroll
-    for (int w = 0; w < kAcceptWarps; ++w)
-      if (sh.red_f[w] > v || (sh.red_f[w] == v && sh.red_i[w] < i)) { v = sh.red_f[w]; i = sh.red_i[w]; }
-    Slot mine;
-    mine.a = 0.0; mine.b = 0.0; mine.f = v; mine.i = i; mine.j = any_bad;
-    cluster_gather(cl, sh, mine, C, kred, all);
-  }
-  float M = -INFINITY;
-  int am = INT_MAX, gbad = 0;
-  for (int r = 0; r < C; ++r) {
-    gbad |= all[r].j;
-    if (all[r].f > M || (all[r].f == M && all[r].i < am)) { M = all[r].f; am = all[r].i; }
-  }
-
-  if (gbad) {
-    d.token = kNonFiniteRow;
-  } else if (greedy) {
-    if (rank == 0) {
+      for (int w = 0; w < kAcceptWarps; ++w)
+        if (sh.red_f[w] > v || (sh.red_f[w] == v && sh.red_i[w] < i)) { v = sh.red_f[w]; i = sh.red_i[w]; }
+      Slot mine;
+      mine.a = 0.0; mine.b = 0.0; mine.f = v; mine.i = i; mine.j = any_bad;
+      cluster_gather(cl, sh, mine, C, kred, all);
+    }
+    int am = INT_MAX;
+    for (int r = 0; r < C; ++r) {
+      gbad |= all[r].j;
+      if (all[r].f > M || (all[r].f == M && all[r].i < am)) { M = all[r].f; am = all[r].i; }
+    }
+    if (gbad) {
+      d.token = kNonFiniteRow;
+    } else if (rank == 0) {
       d.child = first_child_with_token(par, tok, c, n, am, sh);
       d.token = (d.child >= 0) ? -1 : am;
     }
-  } else {
-    // ---- pass B: unnormalised softmax weights e_t in the row frame
-    const double k_d = 1.4426950408889634 / static_cast<double>(p.tau);
-    Frame f;
-    f.k = static_cast<float>(k_d);
-    f.zoff = -M * f.k;
-    f.inv_s = 1.f;
-    f.c = 0.f;
-    f.resid = false;
-    float* seg_w = sh.seg_a;
-    float* seg_r = sh.seg_b;
-    const double tot = weight_pass<false>(zr, nullptr, zvec, false, V, seg0, nloc, f, seg_w, sh);
+  }
+  const double k_d = 1.4426950408889634 / static_cast<double>(p.tau);
+  Frame f;
+  f.k = static_cast<float>(k_d);
+  f.inv_s = 1.f;
+  f.c = 0.f;
+  f.resid = false;
+  if (!greedy) {
+    // ---- one pass: per-segment maximum m_s and sum of 2^((z - m_s) k),
+    // finiteness (and q >= 0); the row frame follows from the gathered
+    // per-CTA maxima
+    bool bad = false;
+    float nf = 0.f;                 // x * 0 turns any non-finite x into NaN
+    float qmin = 0.f;
+    float wmax = -INFINITY;         // running maximum of this warp's segments
+    const float k = f.k;
+    stream_pass(st, -FLT_MAX, [&](int sl, int, const float4 (&v)[4], const float4 (&qv)[4]) {
+      float m = -FLT_MAX;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        m = fmaxf(fmaxf(m, v[kk].x), fmaxf(v[kk].y, fmaxf(v[kk].z, v[kk].w)));
+        nf = fmaf(v[kk].x, 0.f, nf); nf = fmaf(v[kk].y, 0.f, nf);
+        nf = fmaf(v[kk].z, 0.f, nf); nf = fmaf(v[kk].w, 0.f, nf);
+        if (read_q) {
+          qmin = fminf(qmin, fminf(fminf(qv[kk].x, qv[kk].y), fminf(qv[kk].z, qv[kk].w)));
+          nf = fmaf(qv[kk].x, 0.f, nf); nf = fmaf(qv[kk].y, 0.f, nf);
+          nf = fmaf(qv[kk].z, 0.f, nf); nf = fmaf(qv[kk].w, 0.f, nf);
+        }
+      }
+      m = warp_max(m);
+      wmax = fmaxf(wmax, m);
+      const float off = -m * k;
+      float g = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        g += ex2_approx(fmaf(v[kk].x, k, off)) + ex2_approx(fmaf(v[kk].y, k, off));
+        g += ex2_approx(fmaf(v[kk].z, k, off)) + ex2_approx(fmaf(v[kk].w, k, off));
+      }
+      g = warp_sum_f(g);
+      if (lane == 0) { sh.seg_b[sl] = m; sh.seg_a[sl] = g; }
+    });
+    if (nf != nf || qmin < 0.f) bad = true;
+    if (lane == 0) sh.red_f[warp] = wmax;
+    const int any_bad = __syncthreads_or(bad ? 1 : 0);
+    // this CTA's maximum and its sum in that frame
+    float mr = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kAcceptWarps; ++w) mr = fmaxf(mr, sh.red_f[w]);
+    double sr = 0.0;
+    for (int sl = tid; sl < nloc; sl += blockDim.x)
+      sr += static_cast<double>(sh.seg_a[sl]) * exp2(static_cast<double>(sh.seg_b[sl] - mr) * k_d);
+    sr = block_sum_d(sr, sh);
     {
       Slot mine;
-      mine.a = tot; mine.b = 0.0; mine.f = 0.f; mine.i = 0; mine.j = 0;
+      mine.a = sr; mine.b = 0.0; mine.f = mr; mine.i = 0; mine.j = any_bad;
       cluster_gather(cl, sh, mine, C, kred, all);
     }
-    double ssum = 0.0;
-    for (int r = 0; r < C; ++r) { ssum += all[r].a; sh.rank_tot[r] = all[r].a; }
-    __syncthreads();
+    for (int r = 0; r < C; ++r) { gbad |= all[r].j; M = fmaxf(M, all[r].f); }
+    if (gbad) d.token = kNonFiniteRow;
+    else {
+      for (int r = 0; r < C; ++r) {
+        const double tr = (all[r].f == -INFINITY) ? 0.0 : all[r].a * exp2(static_cast<double>(all[r].f - M) * k_d);
+        ssum += tr;
+        if (tid == 0) sh.rank_tot[r] = tr;
+      }
+      // segment sums in the row frame
+      for (int sl = tid; sl < nloc; sl += blockDim.x)
+        sh.seg_a[sl] = sh.seg_a[sl] * ex2_approx((sh.seg_b[sl] - M) * k);
+      __syncthreads();
+    }
+  }
+
+  if (!greedy && !gbad) {
+    f.zoff = -M * f.k;
+    float* seg_w = sh.seg_a;
+    float* seg_r = sh.seg_b;
     const double inv_s = 1.0 / ssum;
     // the weights e_t carry the fp32 frame offset zoff; point values use the
     // same offset in fp64: p(x) = 2^(z_x k + zoff) / s
@@ -522,31 +765,35 @@ accept_node_kernel(AcceptParams p) {
     if (read_q) {
       const float* q = qr;
       int kk = 0;   // child ordinal = draw index
-      for (int base = c + 1; base < n && !decided; base += blockDim.x) {
-        const int j = base + tid;
-        const bool is = (j < n) && par[j] == c;
-        const unsigned m = __ballot_sync(0xffffffffu, is);
-        if (lane == 0) sh.red_i[warp] = __popc(m);
-        __syncthreads();
-        if (tid == 0) {
-          int acc = 0;
-          for (int w = 0; w < kAcceptWarps; ++w) { sh.wofs[w] = acc; acc += sh.red_i[w]; }
-          sh.bc_int[3] = acc;
+      for (int base = c + 1, win = 0; base < n && !decided; base += blockDim.x, ++win) {
+        int cnt = cnt0;           // the first window was listed before the first pass
+        if (win > 0) {
+          const int j = base + tid;
+          const bool is = (j < n) && par[j] == c;
+          const unsigned m = __ballot_sync(0xffffffffu, is);
+          if (lane == 0) sh.red_i[warp] = __popc(m);
+          __syncthreads();
+          if (tid == 0) {
+            int acc = 0;
+            for (int w = 0; w < kAcceptWarps; ++w) { sh.wofs[w] = acc; acc += sh.red_i[w]; }
+            sh.bc_int[3] = acc;
+          }
+          __syncthreads();
+          if (is) sh.clist[sh.wofs[warp] + __popc(m & ((1u << lane) - 1u))] = j;
+          cnt = sh.bc_int[3];
+          __syncthreads();
         }
-        __syncthreads();
-        if (is) sh.clist[sh.wofs[warp] + __popc(m & ((1u << lane) - 1u))] = j;
-        const int cnt = sh.bc_int[3];
-        __syncthreads();
         for (int ci = 0; ci < cnt && !decided; ++ci, ++kk) {
           const int jc = sh.clist[ci];
-          const int x = tok[jc];
+          const int x = (win == 0) ? sh.ctok[ci] : tok[jc];
           if (x < 0 || x >= V) continue;
-          const double px = exp2(static_cast<double>(zr[x]) * k_f + zoff_d) * inv_s;
-          const double qx = static_cast<double>(q[x]);
+          const float zx = (win == 0) ? sh.cz[ci] : zr[x];
+          const double px = exp2(static_cast<double>(zx) * k_f + zoff_d) * inv_s;
+          const double qx = static_cast<double>((win == 0) ? sh.cq[ci] : q[x]);
           const double num = px - cpar * qx;
           const double rx = num > 0.0 ? num / D : 0.0;
           const double ratio = qx > 0.0 ? rx / qx : (rx > 0.0 ? INFINITY : 0.0);
-          const double u = accept_uniform(p.seed, p.step, b, c, kk, kTagChild);
+          const double u = (win == 0) ? sh.cu[ci] : accept_uniform(p.seed, p.step, b, c, kk, kTagChild);
           if (isfinite(ratio)) margin = fmin(margin, fabs(u - ratio));
           if (u < ratio) {
             d.child = jc;
@@ -559,7 +806,7 @@ accept_node_kernel(AcceptParams p) {
           fr.inv_s = static_cast<float>(inv_s);
           fr.c = static_cast<float>(cn);
           fr.resid = true;
-          const double S_loc = weight_pass<true>(zr, q, zvec, qvec, V, seg0, nloc, fr, seg_r, sh);
+          const double S_loc = weight_pass(st, fr, seg_r, sh);
           Slot ms;
           ms.a = S_loc; ms.b = 0.0; ms.f = 0.f; ms.i = 0; ms.j = 0;
           cluster_gather(cl, sh, ms, C, kred, all);
@@ -577,8 +824,7 @@ accept_node_kernel(AcceptParams p) {
     if (!decided) {
       // inverse-CDF sample over the current weights: find the CTA whose
       // slice holds the crossing, search inside it, gather the result
-      const int tag = specsample ? kTagResidual : kTagSpecExec;
-      const double u = accept_uniform(p.seed, p.step, b, c, 0, tag);
+      const double u = sh.bc_dbl[3];
       double W = 0.0;
       for (int r = 0; r < C; ++r) W += sh.rank_tot[r];
       const double target = u * W;
@@ -627,7 +873,9 @@ accept_node_kernel(AcceptParams p) {
     __syncthreads();
     if (sh.bc_int[2]) {
       __threadfence();
-      accept_walk(p, b, n, sh);
+      // the rings are idle now: their shared memory holds the decisions
+      accept_walk(p, b, n, sh, reinterpret_cast<AcceptDec*>(ring_smem),
+                  static_cast<int>(kRingBytes / sizeof(AcceptDec)));
       if (tid == 0) p.ticket[b] = 0;           // ready for the next call
     }
   }
@@ -676,10 +924,13 @@ cudaError_t launch_accept(const tv_accept_args* a, int mode, void* ws, cudaStrea
   p.C = C;
   p.seg_per_cta = (nseg + C - 1) / C;
   const int rows = a->T > 0 ? a->T : 1;        // T == 0: one cluster writes the empty result
+  cudaError_t e = cudaFuncSetAttribute(accept_node_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kRingBytes));
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rows * C, a->B, 1);
   cfg.blockDim = dim3(kAcceptThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = kRingBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -688,7 +939,7 @@ cudaError_t launch_accept(const tv_accept_args* a, int mode, void* ws, cudaStrea
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, accept_node_kernel, p);
+  e = cudaLaunchKernelEx(&cfg, accept_node_kernel, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -10,10 +10,15 @@
 // and a cursor; the candidate set of a round is the union of the lists from
 // their cursors.  (Tokens past the remaining budget can never be taken.)
 //
-//   expand_rows_kernel   one CTA per row: lse of the row and a radix select
-//                        of its top-K logits (three histogram passes on the
-//                        order-preserving 32-bit key), then a bitonic sort
-//                        of those K into the node's list;
+//   expand_rows_kernel   one CTA per row: the row's maximum and minimum,
+//                        then its lse with a histogram of 2048 value bins
+//                        over [min, max] (monotone in the logit, so the
+//                        boundary bin of the top K follows by a prefix
+//                        count), then the bins above the boundary plus an
+//                        exact sort of the boundary bin's members, and a
+//                        bitonic sort of the K into the node's list (a
+//                        boundary bin too crowded for shared memory falls
+//                        back to a radix select on the 32-bit key);
 //   expand_merge_kernel  one CTA: repeatedly take the best s <= 128
 //                        candidates of the union.  The s-th best list head
 //                        bounds the s-th best candidate, so only the <= s
@@ -45,7 +50,7 @@ constexpr int kMergeThreads = 1024;
 constexpr int kMergeWarps = kMergeThreads / kWarp;
 constexpr int kMergeStep = 128;                     // nodes taken per sub-step
 constexpr int kMergeCap = kMergeStep * kMergeStep;  // candidate capacity
-constexpr int kSegE = 128;
+constexpr int kCandCap = 4096;                      // boundary-bin candidates in shared memory
 
 __host__ __device__ inline int64_t expand_kcap(int budget, int V) {
   int64_t k = budget - 1;
@@ -140,14 +145,139 @@ __device__ void find_rank_bin(const uint32_t* hist, int nbins, int rank, int* bi
   __syncthreads();
 }
 
+// Ascending bitonic sort of P (a power of two, 2 <= P) keys in shared
+// memory by the whole block.  Stages whose partners lie within a 64-key
+// block run in registers (warp w, lane l holds keys 64b + l and 64b + 32 + l
+// of its blocks b): the partner 32 apart is the thread's other key, closer
+// partners come by shuffle.  Wider stages compare in shared memory.
+__device__ __forceinline__ uint64_t cas_u64(uint64_t v, uint64_t pv, bool keep_min) {
+  return keep_min ? (v < pv ? v : pv) : (v > pv ? v : pv);
+}
+
+__device__ void bitonic_block64(uint64_t* buf, int P, int k, int jmax) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
+  for (int blk = warp; blk * 64 < P; blk += nw) {
+    const int i0 = blk * 64 + lane, i1 = i0 + 32;
+    uint64_t v0 = buf[i0], v1 = buf[i1];
+    for (int kk = (k <= 64 ? 2 : k); kk <= (k <= 64 ? 64 : k); kk <<= 1) {
+      const int jtop = (k <= 64) ? (kk >> 1) : jmax;
+      for (int j = jtop; j > 0; j >>= 1) {
+        if (kk > P) break;
+        const bool up0 = (i0 & kk) == 0, up1 = (i1 & kk) == 0;
+        if (j == 32) {
+          // partners i0 and i1 = i0 + 32: i0 is the lower index
+          const uint64_t a = v0, b = v1;
+          v0 = cas_u64(a, b, up0);
+          v1 = cas_u64(b, a, !up1);
+        } else {
+          const uint64_t p0 = __shfl_xor_sync(0xffffffffu, v0, j);
+          const uint64_t p1 = __shfl_xor_sync(0xffffffffu, v1, j);
+          const bool low0 = (i0 & j) == 0, low1 = (i1 & j) == 0;
+          v0 = cas_u64(v0, p0, low0 == up0);
+          v1 = cas_u64(v1, p1, low1 == up1);
+        }
+      }
+      if (k > 64) break;
+    }
+    buf[i0] = v0;
+    buf[i1] = v1;
+  }
+}
+
+__device__ void bitonic_sort_u64(uint64_t* buf, int P) {
+  const int tid = threadIdx.x;
+  if (P < 64) {
+    // small: plain shared-memory stages
+    for (int k = 2; k <= P; k <<= 1)
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = tid; i < P; i += blockDim.x) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const uint64_t a = buf[i], b = buf[ixj];
+            const bool up = (i & k) == 0;
+            if ((a > b) == up) { buf[i] = b; buf[ixj] = a; }
+          }
+        }
+        __syncthreads();
+      }
+    return;
+  }
+  // k = 2 .. 64 entirely in registers
+  bitonic_block64(buf, P, 64, 32);
+  __syncthreads();
+  for (int k = 128; k <= P; k <<= 1) {
+    for (int j = k >> 1; j >= 64; j >>= 1) {
+      for (int i = tid; i < P; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint64_t a = buf[i], b = buf[ixj];
+          const bool up = (i & k) == 0;
+          if ((a > b) == up) { buf[i] = b; buf[ixj] = a; }
+        }
+      }
+      __syncthreads();
+    }
+    bitonic_block64(buf, P, k, 32);
+    __syncthreads();
+  }
+}
+
 // ------------------------------------------------------------ row kernel
+
+__device__ __forceinline__ float warp_min_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// The elements of a row pass: iteration it of a thread covers elements
+// 4 (it * blockDim + tid) .. + 3; every thread runs the same number of
+// iterations (ballots stay warp-uniform), four loads in flight per batch.
+template <class F>
+__device__ __forceinline__ void row_pass(const float* row, int V, bool vec, F&& f) {
+  const int tid = threadIdx.x;
+  const int per = 4 * static_cast<int>(blockDim.x);
+  const int iters = (V + per - 1) / per;
+  for (int it0 = 0; it0 < iters; it0 += 4) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e0 = ((it0 + u) * static_cast<int>(blockDim.x) + tid) * 4;
+      v[u] = (it0 + u < iters) ? load4(row, e0, V, vec, 0.f) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (it0 + u >= iters) break;
+      const int e0 = ((it0 + u) * static_cast<int>(blockDim.x) + tid) * 4;
+      const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) f(e0 + k, xs[k], e0 + k < V);
+    }
+  }
+}
+
+// Appends the lanes' flagged 64-bit entries at buf[*count ..] (one shared
+// atomic per warp); entries past cap are dropped (the count still grows).
+__device__ __forceinline__ void warp_append(bool take, uint64_t v, uint64_t* buf, int* count, int cap) {
+  const int lane = threadIdx.x & 31;
+  const unsigned m = __ballot_sync(0xffffffffu, take);
+  if (m == 0u) return;
+  int off = 0;
+  if (lane == 0) off = atomicAdd(count, __popc(m));
+  off = __shfl_sync(0xffffffffu, off, 0);
+  if (take) {
+    const int pos = off + __popc(m & ((1u << lane) - 1u));
+    if (pos < cap) buf[pos] = v;
+  }
+}
 
 __global__ void __launch_bounds__(kRowThreads)
 expand_rows_kernel(ExpandParams p) {
   extern __shared__ __align__(16) unsigned char dsm[];
   __shared__ RowShared sh;
   __shared__ uint32_t hist[2048];
-  __shared__ int s_count;
+  __shared__ int s_count, s_cand;
   const int r = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int node = p.row_node[r];
@@ -168,66 +298,47 @@ expand_rows_kernel(ExpandParams p) {
   if (K <= 0) return;
   const float* row = p.logits + static_cast<int64_t>(r) * p.ld;
   const bool vec = (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
-  const int nseg = (V + kSegE - 1) / kSegE;
   const int P = 1 << (32 - __clz(K - 1 | 1));      // next power of two >= K (>= 2)
   uint64_t* sbuf = reinterpret_cast<uint64_t*>(dsm);
-  double* seg_s = reinterpret_cast<double*>(sbuf + P);
-  float* seg_m = reinterpret_cast<float*>(seg_s + nseg);
+  uint64_t* cbuf = sbuf + P;                         // boundary-bin candidates
   const double invtau = 1.0 / static_cast<double>(p.tau);
 
-  for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
-  // pass 1: segment max / exp sums, finiteness, histogram of the top 11 key bits
+  // pass 1: finiteness, row maximum and minimum
   bool bad = false;
-  float lmax = -INFINITY;
-  for (int s = warp; s < nseg; s += kRowWarps) {
-    const int e0 = s * kSegE + lane * 4;
-    const float4 v = load4(row, e0, V, vec, 0.f);
-    const float xs[4] = {v.x, v.y, v.z, v.w};
-    float m4 = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      if (e0 + k < V) {
-        if (!isfinite(xs[k])) bad = true;
-        else {
-          m4 = fmaxf(m4, xs[k]);
-          atomicAdd(&hist[zdesc_key(xs[k]) >> 21], 1u);
-        }
-      }
-    const float wm = warp_max(m4);
-    double a = 0.0;
-    // double-precision exponentials: the row's lse enters every cumulative
-    // score, and cross-row ranks must not move by more than fp64 rounding
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      if (e0 + k < V && isfinite(xs[k]))
-        a += exp((static_cast<double>(xs[k]) - static_cast<double>(wm)) * invtau);
-    a = warp_sum(a);
-    if (lane == 0) { seg_m[s] = wm; seg_s[s] = a; }
-    lmax = fmaxf(lmax, wm);
-  }
+  float lmax = -INFINITY, lmin = INFINITY;
+  row_pass(row, V, vec, [&](int, float x, bool in) {
+    if (!in) return;
+    if (!isfinite(x)) bad = true;
+    else { lmax = fmaxf(lmax, x); lmin = fminf(lmin, x); }
+  });
   const int any_bad = __syncthreads_or(bad ? 1 : 0);
   if (any_bad) {
     if (tid == 0) set_status(p.status, TV_DEV_NONFINITE);
     return;
   }
-  // row maximum and lse = M/tau + log sum exp((z - M)/tau)
-  float M = warp_max(lmax);
-  if (lane == 0) sh.red_f[warp] = M;
+  lmax = warp_max(lmax);
+  lmin = warp_min_f(lmin);
+  if (lane == 0) { sh.red_f[warp] = lmax; sh.red_d[warp] = static_cast<double>(lmin); }
+  for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  if (warp == 0) {
-    float t = (lane < kRowWarps) ? sh.red_f[lane] : -INFINITY;
-    t = warp_max(t);
-    if (lane == 0) sh.red_f[0] = t;
-  }
+  float M = -INFINITY, mn = INFINITY;
+  for (int w = 0; w < kRowWarps; ++w) { M = fmaxf(M, sh.red_f[w]); mn = fminf(mn, static_cast<float>(sh.red_d[w])); }
   __syncthreads();
-  M = sh.red_f[0];
-  double part = 0.0;
-  for (int s = tid; s < nseg; s += blockDim.x)
-    part += seg_s[s] * exp((static_cast<double>(seg_m[s]) - static_cast<double>(M)) * invtau);
-  part = warp_sum(part);
-  __syncthreads();
-  if (lane == 0) sh.red_d[warp] = part;
+  // pass 2: value bins (M - z) * 2047 / (M - min), non-decreasing as z
+  // falls, so bin order is rank order; and the row's sum of exponentials
+  const float range = M - mn;
+  const float sc = (range > 0.f && isfinite(range)) ? 2047.f / range : 0.f;
+  double es = 0.0;
+  row_pass(row, V, vec, [&](int, float x, bool in) {
+    if (!in) return;
+    const int bin = static_cast<int>(fminf((M - x) * sc, 2047.f));
+    atomicAdd(&hist[bin], 1u);
+    // double-precision exponentials: the row's lse enters every cumulative
+    // score, and cross-row ranks must not move by more than fp64 rounding
+    es += exp((static_cast<double>(x) - static_cast<double>(M)) * invtau);
+  });
+  es = warp_sum(es);
+  if (lane == 0) sh.red_d[warp] = es;
   __syncthreads();
   if (warp == 0) {
     double t = (lane < kRowWarps) ? sh.red_d[lane] : 0.0;
@@ -237,91 +348,118 @@ expand_rows_kernel(ExpandParams p) {
   __syncthreads();
   const double lse = static_cast<double>(M) * invtau + log(sh.bcd[0]);
 
-  // radix select of the K-th smallest descending key (11 + 11 + 10 bits)
   int b1, before;
   find_rank_bin(hist, 2048, K, &b1, &before, sh);
-  int need = K - before;
-  for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
-  for (int e = tid; e < V; e += blockDim.x) {
-    const uint32_t k = zdesc_key(__ldg(row + e));
-    if ((k >> 21) == static_cast<uint32_t>(b1)) atomicAdd(&hist[(k >> 10) & 0x7FFu], 1u);
-  }
-  __syncthreads();
-  int b2;
-  find_rank_bin(hist, 2048, need, &b2, &before, sh);
-  need -= before;
-  const uint32_t pre2 = (static_cast<uint32_t>(b1) << 11) | static_cast<uint32_t>(b2);
-  for (int i = tid; i < 1024; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
-  for (int e = tid; e < V; e += blockDim.x) {
-    const uint32_t k = zdesc_key(__ldg(row + e));
-    if ((k >> 10) == pre2) atomicAdd(&hist[k & 0x3FFu], 1u);
-  }
-  __syncthreads();
-  int b3;
-  find_rank_bin(hist, 1024, need, &b3, &before, sh);
-  need -= before;                                    // ties at theta to take
-  const uint32_t theta = (pre2 << 10) | static_cast<uint32_t>(b3);
-  const int n_eq = static_cast<int>(hist[b3]);
-
-  // collect: keys below theta, then the first `need` ties by token index
-  if (tid == 0) s_count = 0;
-  __syncthreads();
-  for (int e = tid; e < V; e += blockDim.x) {
-    const uint32_t k = zdesc_key(__ldg(row + e));
-    if (k < theta || (k == theta && n_eq == need)) {
-      const int pos = atomicAdd(&s_count, 1);
-      if (pos < K) sbuf[pos] = (static_cast<uint64_t>(k) << 32) | static_cast<uint32_t>(e);
+  const int n1 = static_cast<int>(hist[b1]);
+  const int need = K - before;                     // taken from the boundary bin
+  if (n1 <= kCandCap) {
+    // pass 3: the bins above the boundary go to the list, the boundary bin
+    // to the candidates, whose exact order (key, token) decides the rest
+    if (tid == 0) { s_count = 0; s_cand = 0; }
+    __syncthreads();
+    row_pass(row, V, vec, [&](int e, float x, bool in) {
+      const int bin = in ? static_cast<int>(fminf((M - x) * sc, 2047.f)) : 2048;
+      const uint64_t v = (static_cast<uint64_t>(zdesc_key(x)) << 32) | static_cast<uint32_t>(e);
+      warp_append(bin < b1, v, sbuf, &s_count, K);
+      warp_append(bin == b1, v, cbuf, &s_cand, kCandCap);
+    });
+    __syncthreads();
+    const int nc = min(s_cand, kCandCap);
+    const int Pc = 1 << (32 - __clz(nc - 1 | 1));
+    for (int i = nc + tid; i < Pc; i += blockDim.x) cbuf[i] = ~0ull;
+    __syncthreads();
+    bitonic_sort_u64(cbuf, Pc);
+    for (int i = tid; i < need; i += blockDim.x) sbuf[before + i] = cbuf[i];
+    __syncthreads();
+  } else {
+    // a crowded boundary bin: radix select on the 32-bit key instead
+    // (11 + 11 + 10 bits), then the keys below the threshold and the first
+    // ties by token index
+    __syncthreads();
+    for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    row_pass(row, V, vec, [&](int, float x, bool in) {
+      if (in) atomicAdd(&hist[zdesc_key(x) >> 21], 1u);
+    });
+    __syncthreads();
+    int kb1, kbefore;
+    find_rank_bin(hist, 2048, K, &kb1, &kbefore, sh);
+    int kneed = K - kbefore;
+    for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int e = tid; e < V; e += blockDim.x) {
+      const uint32_t k = zdesc_key(__ldg(row + e));
+      if ((k >> 21) == static_cast<uint32_t>(kb1)) atomicAdd(&hist[(k >> 10) & 0x7FFu], 1u);
     }
-  }
-  __syncthreads();
-  if (n_eq != need) {
-    // ordered pass over the row for the ties
-    int taken = 0;
-    for (int base = 0; base < V && taken < need; base += blockDim.x) {
-      const int e = base + tid;
-      const bool is = (e < V) && zdesc_key(__ldg(row + e)) == theta;
-      const unsigned m = __ballot_sync(0xffffffffu, is);
-      if (lane == 0) sh.red_i[warp] = __popc(m);
-      __syncthreads();
-      if (warp == 0) {
-        const int v = (lane < kRowWarps) ? sh.red_i[lane] : 0;
-        int incl = v;
+    __syncthreads();
+    int b2;
+    find_rank_bin(hist, 2048, kneed, &b2, &kbefore, sh);
+    kneed -= kbefore;
+    const uint32_t pre2 = (static_cast<uint32_t>(kb1) << 11) | static_cast<uint32_t>(b2);
+    for (int i = tid; i < 1024; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int e = tid; e < V; e += blockDim.x) {
+      const uint32_t k = zdesc_key(__ldg(row + e));
+      if ((k >> 10) == pre2) atomicAdd(&hist[k & 0x3FFu], 1u);
+    }
+    __syncthreads();
+    int b3;
+    find_rank_bin(hist, 1024, kneed, &b3, &kbefore, sh);
+    const int need3 = kneed - kbefore;                 // ties at theta to take
+    const uint32_t theta = (pre2 << 10) | static_cast<uint32_t>(b3);
+    const int n_eq = static_cast<int>(hist[b3]);
+
+    // collect: keys below theta, then the first `need` ties by token index
+    if (tid == 0) s_count = 0;
+    __syncthreads();
+    for (int base = warp * 32; base < V; base += blockDim.x) {
+      const int e = base + lane;
+      const uint32_t k = (e < V) ? zdesc_key(__ldg(row + e)) : ~0u;
+      const bool take = (e < V) && (k < theta || (k == theta && n_eq == need3));
+      const unsigned m = __ballot_sync(0xffffffffu, take);
+      int off = 0;
+      if (lane == 0 && m) off = atomicAdd(&s_count, __popc(m));
+      off = __shfl_sync(0xffffffffu, off, 0);
+      if (take) {
+        const int pos = off + __popc(m & ((1u << lane) - 1u));
+        if (pos < K) sbuf[pos] = (static_cast<uint64_t>(k) << 32) | static_cast<uint32_t>(e);
+      }
+    }
+    __syncthreads();
+    if (n_eq != need3) {
+      // ordered pass over the row for the ties
+      int taken = 0;
+      for (int base = 0; base < V && taken < need3; base += blockDim.x) {
+        const int e = base + tid;
+        const bool is = (e < V) && zdesc_key(__ldg(row + e)) == theta;
+        const unsigned m = __ballot_sync(0xffffffffu, is);
+        if (lane == 0) sh.red_i[warp] = __popc(m);
+        __syncthreads();
+        if (warp == 0) {
+          const int v = (lane < kRowWarps) ? sh.red_i[lane] : 0;
+          int incl = v;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int t = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t;
+          for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+          }
+          if (lane < kRowWarps) sh.red_i[lane] = incl - v;
+          if (lane == 31) sh.bc[3] = incl;
         }
-        if (lane < kRowWarps) sh.red_i[lane] = incl - v;
-        if (lane == 31) sh.bc[3] = incl;
+        __syncthreads();
+        const int rank = taken + sh.red_i[warp] + __popc(m & ((1u << lane) - 1u));
+        if (is && rank < need3) {
+          const int pos = atomicAdd(&s_count, 1);
+          if (pos < K) sbuf[pos] = (static_cast<uint64_t>(theta) << 32) | static_cast<uint32_t>(e);
+        }
+        taken += sh.bc[3];
+        __syncthreads();
       }
-      __syncthreads();
-      const int rank = taken + sh.red_i[warp] + __popc(m & ((1u << lane) - 1u));
-      if (is && rank < need) {
-        const int pos = atomicAdd(&s_count, 1);
-        if (pos < K) sbuf[pos] = (static_cast<uint64_t>(theta) << 32) | static_cast<uint32_t>(e);
-      }
-      taken += sh.bc[3];
-      __syncthreads();
     }
   }
   for (int i = K + tid; i < P; i += blockDim.x) sbuf[i] = ~0ull;
   __syncthreads();
-  // bitonic sort ascending: (z desc, token asc)
-  for (int k = 2; k <= P; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < P; i += blockDim.x) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const uint64_t a = sbuf[i], b = sbuf[ixj];
-          const bool up = (i & k) == 0;
-          if ((a > b) == up) { sbuf[i] = b; sbuf[ixj] = a; }
-        }
-      }
-      __syncthreads();
-    }
-  }
+  bitonic_sort_u64(sbuf, P);
   ListEntry* lst = p.lists + static_cast<int64_t>(node) * p.kcap;
   for (int i = tid; i < K; i += blockDim.x) {
     const uint64_t v = sbuf[i];
@@ -594,11 +732,10 @@ cudaError_t launch_expand_init(const tv_expand_args* a, int root_token, cudaStre
 cudaError_t launch_expand(const tv_expand_args* a, cudaStream_t stream) {
   ExpandParams p = make_params(a);
   if (a->R > 0) {
-    const int nseg = (a->V + kSegE - 1) / kSegE;
     const int K = static_cast<int>(expand_kcap(a->budget, a->V));
     int P = 2;
     while (P < K) P <<= 1;
-    const size_t smem = static_cast<size_t>(P) * 8 + static_cast<size_t>(nseg) * 12 + 16;
+    const size_t smem = (static_cast<size_t>(P) + kCandCap) * sizeof(uint64_t);
     cudaError_t e = cudaFuncSetAttribute(expand_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
