@@ -43,6 +43,35 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
 
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic.txt")
+KERNEL_SOURCES = {
+    "accept_node_kernel": "tree_verification_verify_b200/csrc/accept.cu",
+    "attn_tc_kernel": "tree_verification_verify_b200/csrc/attn_tc.cu",
+    "expand_rows_kernel": "tree_verification_verify_b200/csrc/expand.cu",
+}
+
+
+def measured_traffic(kernel, workload):
+    """DRAM bytes per launch (read + write) of `kernel` on `workload` from the
+    committed ncu summary, or None when there is none or the kernel's source
+    has changed since the counters were taken (the summary records the
+    source's sha1)."""
+    import hashlib
+    try:
+        src = os.path.join(ROOT, KERNEL_SOURCES[kernel])
+        sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
+        for line in open(TRAFFIC_PATH):
+            f = line.split()
+            if len(f) < 4 or f[0].startswith("#"):
+                continue
+            kv = dict(x.split("=", 1) for x in f[2:] if "=" in x)
+            if f[0] == kernel and f[1] == workload and kv.get("source_sha1") == sha:
+                return float(kv["dram_bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
 def peaks():
     try:
         with open(PEAKS_PATH) as f:
@@ -499,22 +528,32 @@ def main():
         roof = {"kernel": "tree_expand_topb (16 rounds: row + merge launches)", "bound": "hbm",
                 "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
                 "traffic": None, "peak_source": src, "algorithmic_bytes": step.expand_bytes}
+        tk = "expand_rows_kernel"
     elif ms_acc >= ms_attn:
         achieved = step.accept_bytes / (ms_acc * 1e-3) / 1e9
-        roof = {"kernel": "tree_accept (node + walk launches)", "bound": "hbm", "achieved": round(achieved, 1),
+        roof = {"kernel": "accept_node_kernel (tree_accept: one launch)", "bound": "hbm",
+                "achieved": round(achieved, 1),
                 "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
                 "peak_source": src, "algorithmic_bytes": step.accept_bytes}
+        tk = "accept_node_kernel"
     else:
         if step.attn_bytes / (hbm * 1e9) >= step.attn_flops / (bf16 * 1e12):
             achieved = step.attn_bytes / (ms_attn * 1e-3) / 1e9
             roof = {"kernel": "tree_verify_attn (all launches)", "bound": "hbm", "achieved": round(achieved, 1),
                     "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
                     "peak_source": src, "algorithmic_bytes": step.attn_bytes}
+            tk = "attn_tc_kernel"
         else:
             achieved = step.attn_flops / (ms_attn * 1e-3) / 1e12
             roof = {"kernel": "tree_verify_attn (all launches)", "bound": "tensor", "achieved": round(achieved, 2),
                     "peak": bf16, "unit": "TFLOP/s", "frac": round(achieved / bf16, 4), "traffic": None,
                     "peak_source": src, "algorithmic_flops": step.attn_flops}
+            tk = "attn_tc_kernel"
+    if step.attn_path != 1 and tk == "attn_tc_kernel":
+        roof["kernel"] = "tree_verify_attn (all launches)"
+    else:
+        roof["traffic"] = measured_traffic(tk, step.name)
+        roof["traffic_source"] = "profiles/traffic.txt (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
     line = {
         "metric": METRIC, "value": tokens / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
