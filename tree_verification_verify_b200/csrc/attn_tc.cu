@@ -68,7 +68,9 @@ constexpr uint32_t kSmemPar = kSmemV + kVS * kTileBytes;  // parent[] (u16)
 constexpr uint32_t kSmemUL = kSmemPar + kMaxT * 2;        // U: slot -> node (u16)
 constexpr uint32_t kSmemUP = kSmemUL + kMaxT * 2;         // U: slot -> parent's slot (u16)
 constexpr uint32_t kSmemBytes = kSmemUP + kMaxT * 2;      // 216 KB
-constexpr uint32_t kSmemInbox = kSmemK;                   // merge: fp32 O rows pushed by the cluster
+constexpr uint32_t kSmemInbox = kSmemK;                   // merge: fp32 O rows copied in by the cluster
+constexpr uint32_t kSmemStage = kSmemV;                   // merge: this CTA's fp32 O rows (idle V ring)
+constexpr int kMaxInboxRows = 144;                        // max over C of C * per (per = 4 * ceil(128 / 4C))
 constexpr uint32_t kTmemCols = 512;                       // S0, S1, O (128 each)
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr uint32_t kWaitLimit = 1u << 22;
@@ -76,8 +78,9 @@ constexpr uint32_t kDrainLimit = 1u << 20;
 constexpr uint16_t kRootMark = 0xFFFEu;   // parent[] entry of a well-formed root
 constexpr uint16_t kBadMark = 0xFFFFu;    // malformed parent (or no parent slot)
 
-static_assert(kSmemInbox + (kRows + kMaxCluster) * kD * 4 <= kSmemK + kKS * kTileBytes,
+static_assert(kSmemInbox + kMaxInboxRows * kD * 4 <= kSmemK + kKS * kTileBytes,
               "the merge inbox fits the K ring");
+static_assert(kSmemStage + kRows * kD * 4 <= kSmemV + kVS * kTileBytes, "the merge stage fits the V ring");
 
 struct Bars {
   uint64_t q_full;
@@ -92,8 +95,9 @@ struct Bars {
   uint32_t bm[kMaxT / 32];          // node bitmap of U
   int pre[kMaxT / 32];              // marked nodes below each bitmap word
   int node_ok[kRows];               // root path of the tile's node is well formed
-  float in_lse[kRows + kMaxCluster]; // merge inbox: log2-sum-exp of row (chunk, row)
-  int in_abort[kMaxCluster];        // merge inbox: the chunk's CTA aborted
+  uint64_t inbox_full;              // the cluster's copies into this CTA's inbox have landed
+  alignas(16) float st_lse[kRows];  // this CTA's rows: log2-sum-exp (NaN: invalid)
+  alignas(16) float in_lse[kMaxInboxRows];  // merge inbox: log2-sum-exp of row (chunk, row)
 };
 
 
@@ -273,6 +277,44 @@ __device__ __forceinline__ int u_slot(const Bars& bars, int a) {
 
 __device__ __forceinline__ uint32_t s_col(int j) { return (j & 1) ? kColS1 : kColS0; }
 
+// Shared-memory address `a` of this CTA mapped to CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t a, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to
+// a cluster peer's, completing on the peer's mbarrier `bar`.
+__device__ __forceinline__ void bulk_s2c(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// Bytes a merging CTA receives from one chunk for `rows` rows: the fp32 O
+// rows and their log-sum-exp (padded to 16 bytes).
+__host__ __device__ constexpr uint32_t merge_bytes(int rows) {
+  return rows > 0 ? static_cast<uint32_t>(rows) * kD * 4 + static_cast<uint32_t>((rows + 3) & ~3) * 4 : 0u;
+}
+
+// Bounded wait (cluster-scope acquire) on phase `parity`; false on expiry.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* b, uint32_t parity) {
+  const uint32_t a = smem_u32(b);
+  for (uint32_t it = 0; it < kWaitLimit; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
 }  // namespace tc
 
 using namespace tc;
@@ -309,6 +351,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   // this thread's query row (softmax warps)
   const int row_node = i0 + tid / G;
   const bool row_valid = tid < kRows && (tid / G) < nodes_here;
+  // rows [c * merge_per, (c + 1) * merge_per) of the tile are merged by CTA c
+  const int merge_per = 4 * ((nodes_here * G + 4 * C - 1) / (4 * C));
 
   // 1024-aligned dynamic shared memory (128B swizzle atoms are 1 KB)
   const uint32_t raw = smem_u32(dsmem_raw);
@@ -326,10 +370,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     for (int s = 0; s < 2; ++s) { mbar_init(&bars.s_full[s], 1); mbar_init(&bars.p_full[s], 4); }
     mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.tree_info, 1);
+    mbar_init(&bars.inbox_full, 1);
     bars.abort = 0;
     bars.nU = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    // the bytes the cluster will copy into this CTA's inbox
+    const int own = max(0, min(merge_per, nodes_here * G - chunk * merge_per));
+    mbar_expect_tx(&bars.inbox_full, static_cast<uint32_t>(C) * merge_bytes(own));
   }
   if (warp == kWarpMma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -342,8 +390,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   __syncthreads();
   fence_after();
   const uint32_t tmem = bars.tmem_base;
-  float orow[kD];              // softmax threads: this row's normalised O
-  float my_lse2 = NAN;         // and its log2-sum-exp
 
   if (warp == kWarpTree) {
     // ------------------------------------------------------------ tree bookkeeping
@@ -546,7 +592,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       }
       if (!ok) {
         // the issued MMAs complete before the TMEM is freed
+        if (s_issued > 1) mbar_drain(&bars.s_full[(s_issued - 2) & 1], ((s_issued - 2) >> 1) & 1);
         if (s_issued > 0) mbar_drain(&bars.s_full[(s_issued - 1) & 1], ((s_issued - 1) >> 1) & 1);
+        if (pv_issued > 1) mbar_drain(&bars.pv_done, (pv_issued - 2) & 1);
         if (pv_issued > 0) mbar_drain(&bars.pv_done, (pv_issued - 1) & 1);
       }
     }
@@ -679,31 +727,44 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       if (lane == 0) mbar_arrive(&bars.p_full[j & 1]);
     }
     // ------------------------------------------------------------ epilogue
+    // The last P V is pv_done's phase ntot - 1.  S(ntot - 1) having landed
+    // only proves P V up to ntot - 3, and a parity wait cannot tell phase
+    // ntot - 1 from ntot - 3: wait for phase ntot - 2 first, then ntot - 1.
+    if (ok && ntot > 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (ntot - 2) & 1, abort));
     if (ok && ntot > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (ntot - 1) & 1, abort));
     fence_after();
     const bool have = ok && l_run > 0.f;
     const float inv = have ? 1.f / l_run : 0.f;
+    // this row's normalised O into the stage (the idle V ring; fp32,
+    // float4 q of row t at q ^ (t & 7)) and its log2-sum-exp
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    float* stage = reinterpret_cast<float*>(gbase + kSmemStage) + tid * kD;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      tmem_ld32(trow + kColO + c * 32, orow + c * 32);
+      float v[32];
+      tmem_ld32(trow + kColO + c * 32, v);
       tmem_wait_ld();
-    }
 #pragma unroll
-    for (int e = 0; e < kD; ++e) orow[e] = have ? orow[e] * inv : 0.f;
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<float4*>(stage + (((c * 8 + q) ^ (tid & 7)) * 4)) =
+            have ? make_float4(v[4 * q] * inv, v[4 * q + 1] * inv, v[4 * q + 2] * inv, v[4 * q + 3] * inv)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     const bool good = !(has_tree && !my_ok) && !bad_len && ok;
-    my_lse2 = !good ? NAN : (l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY);
+    bars.st_lse[tid] = !good ? NAN : (l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY);
+    // the stage is read by bulk copies (async proxy)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (row_valid && has_tree && !my_ok) set_status(p.status, TV_DEV_BAD_PARENT);
     if (bad_len && has_tree && tid == 0) set_status(p.status, TV_DEV_BAD_LEN);
   }
 
   // ------------------------------------------------------------ cluster merge
-  // Row t of the tile is merged by CTA t / per.  Every CTA pushes its rows
-  // (normalised O, fp32) and their log2-sum-exp into the owners' shared
-  // memory (the K rings, idle once all CTAs have left their main loops);
+  // Row t of the tile is merged by CTA t / merge_per.  Once every CTA is
+  // past its main loop (the inboxes are the idle K rings), each CTA copies
+  // its staged rows and their log-sum-exp to the owners with bulk copies
+  // over distributed shared memory, completing on the owner's mbarrier;
   // each owner then merges its rows from local shared memory.
   const int rows_here = nodes_here * G;
-  const int per = (rows_here + C - 1) / C;
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   fence_before();
   cl.sync();                  // every CTA is past its main loop
   fence_after();
@@ -711,41 +772,50 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
-  if (tid < rows_here) {
-    const int owner = tid / per, r = chunk * per + (tid - owner * per);
-    float* dst = cl.map_shared_rank(reinterpret_cast<float*>(gbase + kSmemInbox), owner) + r * kD;
-#pragma unroll
-    for (int q = 0; q < kD / 4; ++q)
-      *reinterpret_cast<float4*>(dst + ((q ^ (r & 7)) * 4)) =
-          make_float4(orow[4 * q], orow[4 * q + 1], orow[4 * q + 2], orow[4 * q + 3]);
-    cl.map_shared_rank(&bars, owner)->in_lse[r] = my_lse2;
+  if (tid == 0) {
+    for (int o = 0; o < C; ++o) {
+      const int r0 = o * merge_per;
+      const int nr = max(0, min(merge_per, rows_here - r0));
+      if (nr == 0) continue;
+      const uint32_t dst_rows = cluster_addr(base + kSmemInbox + (chunk * merge_per) * kD * 4, o);
+      const uint32_t dst_lse = cluster_addr(smem_u32(&bars.in_lse[chunk * merge_per]), o);
+      const uint32_t bar = cluster_addr(smem_u32(&bars.inbox_full), o);
+      bulk_s2c(dst_rows, base + kSmemStage + r0 * kD * 4, static_cast<uint32_t>(nr) * kD * 4, bar);
+      bulk_s2c(dst_lse, smem_u32(&bars.st_lse[r0]), static_cast<uint32_t>((nr + 3) & ~3) * 4, bar);
+    }
   }
-  if (tid < C) cl.map_shared_rank(&bars, tid)->in_abort[chunk] = *abort;
+  // all copies into this CTA have landed
+  const bool inbox_ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bars.inbox_full, 0));
+  if (!inbox_ok) bars.abort = 1;
+  // peers may leave once every CTA has received its rows (so every copy
+  // that reads this CTA's stage is complete); the wait is at the very end
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   if (*abort && tid == 0) set_status(p.status, TV_DEV_TIMEOUT);
-  cl.sync();                  // the pushes have landed
   {
     const float* inbox = reinterpret_cast<const float*>(gbase + kSmemInbox);
-    const int r0 = chunk * per;
-    for (int lt = warp; lt < per && r0 + lt < rows_here; lt += kThreads / 32) {
+    const int r0 = chunk * merge_per;
+    const bool bad_all = !inbox_ok;
+    for (int lt = warp; lt < merge_per && r0 + lt < rows_here; lt += kThreads / 32) {
       const int t = r0 + lt;
-      float lc = -INFINITY;
-      int ab = 0;
-      if (lane < C) {
-        lc = bars.in_lse[lane * per + lt];
-        ab = bars.in_abort[lane];
-      }
-      const bool bad = __any_sync(0xffffffffu, (lc != lc) || ab != 0);
-      if (lc != lc) lc = -INFINITY;
-      const float M = warp_max(lc);
-      const float wl = (lc > -INFINITY) ? ex2_approx(lc - M) : 0.f;
-      const float den = warp_sumf(wl);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      // every lane reads the chunks' log-sum-exp (shared-memory broadcast)
+      float lc[kMaxCluster];
+      float M = -INFINITY;
+      bool bad = bad_all;
 #pragma unroll
       for (int c = 0; c < kMaxCluster; ++c) {
-        const float w = __shfl_sync(0xffffffffu, wl, c);
-        if (c < C && w != 0.f) {
-          const int r = c * per + lt;
-          const float4 v = *reinterpret_cast<const float4*>(inbox + r * kD + ((lane ^ (r & 7)) * 4));
+        lc[c] = (c < C) ? bars.in_lse[c * merge_per + lt] : -INFINITY;
+        bad |= (lc[c] != lc[c]);
+        M = fmaxf(M, lc[c]);
+      }
+      float den = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      const int phys = lane ^ (t & 7);
+#pragma unroll
+      for (int c = 0; c < kMaxCluster; ++c) {
+        const float w = (c < C && lc[c] > -INFINITY) ? ex2_approx(lc[c] - M) : 0.f;
+        den += w;
+        if (w != 0.f) {
+          const float4 v = *reinterpret_cast<const float4*>(inbox + (c * merge_per + lt) * kD + phys * 4);
           acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
           acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
         }
@@ -767,6 +837,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
             okr ? (M + __log2f(den)) * 0.6931471805599453f : NAN;
     }
   }
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ host side
