@@ -299,9 +299,9 @@ TV_API int32_t tv_attn_path(const tv_attn_args* a);
 /* How many kernels tree_verify_attn launches for these arguments (0 when
  * B or T is 0, -1 when the arguments are rejected): 1 for the tensor-core
  * kernel (its prefix chunks are merged inside the launch), 3 on the
- * CUDA-core path (prefix, tree paths, merge), 4 or 5 on
+ * CUDA-core path (prefix, tree paths, merge), 5 or 6 on
  * the block top-k path (block means unless the caller passes them, block
- * selection, sparse prefix, tree paths, merge).  Host only; nothing runs. */
+ * scores, block selection, sparse prefix, tree paths, merge).  Host only; nothing runs. */
 TV_API int32_t tv_attn_launches(const tv_attn_args* a);
 /* Library version, e.g. "treeverify 0.1.0 sm_100a". */
 TV_API const char* tree_verify_version(void);

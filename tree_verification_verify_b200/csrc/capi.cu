@@ -41,7 +41,7 @@ struct AttnPlan {
   bool tc;            // tensor-core prefix kernel
   bool sparse;
   int nchunk, chunk_len, node_tile, nblk_max;
-  size_t off_o, off_lse, off_ok, off_kbar, off_sel, total;
+  size_t off_o, off_lse, off_ok, off_kbar, off_sel, off_scores, total;
 };
 
 tv_status check_attn(const tv_attn_args* a) {
@@ -129,6 +129,8 @@ AttnPlan plan_attn(const tv_attn_args* a) {
       off = align256(off + static_cast<size_t>(a->B) * pl.nblk_max * a->Hkv * a->d * sizeof(float));
     pl.off_sel = off;
     off = align256(off + static_cast<size_t>(a->B) * a->T * a->Hkv * a->sparse_topk * sizeof(int32_t));
+    pl.off_scores = off;
+    off = align256(off + static_cast<size_t>(a->B) * a->T * a->Hkv * pl.nblk_max * sizeof(float));
   }
   pl.total = off;
   return pl;
@@ -153,7 +155,7 @@ extern "C" int32_t tv_attn_launches(const tv_attn_args* a) {
   if (check_attn(a) != TV_OK) return -1;
   if (a->B == 0 || a->T == 0) return 0;
   const AttnPlan pl = plan_attn(a);
-  if (pl.sparse) return (a->k_block_mean ? 0 : 1) + 4;
+  if (pl.sparse) return (a->k_block_mean ? 0 : 1) + 5;
   if (pl.tc) return 1;
   return 3;
 }
@@ -192,6 +194,7 @@ extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws
     p.topk = a->sparse_topk; p.block_size = a->block_size; p.nblk_max = pl.nblk_max;
     p.kbar = a->k_block_mean ? a->k_block_mean : reinterpret_cast<float*>(w + pl.off_kbar);
     p.sel = reinterpret_cast<int32_t*>(w + pl.off_sel);
+    p.scores = reinterpret_cast<float*>(w + pl.off_scores);
     p.sel_out = a->sel_blocks;
     if (!a->k_block_mean) {
       e = launch_block_means(p, reinterpret_cast<float*>(w + pl.off_kbar), s);
