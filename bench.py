@@ -11,11 +11,13 @@ tree tokens per second per layer over all ranks.  Inputs are synthetic
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--config llama3_8b|specexec70b|serving|longctx|longctx_sparse]
 
-Timing: the two calls of a step are captured once into CUDA graphs; W
-untimed warm-up steps, then K steps, each preceded (outside the timed
-region) by a 256 MiB write that flushes the 126 MB L2; each step is
-bracketed by CUDA events on the launching stream, per-call events give the
-per-call durations; the max over ranks is reported.  The e2e figure calls
+Timing: the step's calls are captured once into one CUDA graph (and each
+call into a graph of its own); W untimed warm-up steps, then K steps of the
+one-graph step, each preceded (outside the timed region) by a 256 MiB write
+that flushes the 126 MB L2 and bracketed by CUDA events on the launching
+stream (`ms_per_step`, `value`); then K steps of the per-call graphs with an
+event between calls give the per-call durations (`calls`); the max over
+ranks is reported.  The e2e figure calls
 the Python API directly (no graph), copying the step's inputs from pinned
 host memory and reading the accepted tokens back.  --impl reference times
 the fp64 CPU oracle on a bounded sample of the same workload.
@@ -305,30 +307,47 @@ def capture_graphs(step):
     # capture on the warm-up stream: the binding's per-stream workspace then
     # already exists and nothing is allocated (or zero-filled) in the graph
     graphs = {}
-    for name, fn in (("expand", step.run_expand if step.expand else None),
-                     ("attn", step.run_attn), ("accept", step.run_accept)):
-        if fn is None:
-            continue
+    calls = [(name, fn) for name, fn in (("expand", step.run_expand if step.expand else None),
+                                         ("attn", step.run_attn), ("accept", step.run_accept)) if fn]
+    for name, fn in calls:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=s):
             fn()
         graphs[name] = g
+    # the whole step as one graph (how a caller launches it)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for _, fn in calls:
+            fn()
+    graphs["step"] = g
     torch.cuda.synchronize()
     return graphs
 
 
 def time_steps(step, K, W, world, flush):
+    """K timed steps, each the one-graph step (`step`), then K steps of the
+    per-call graphs with an event between calls (the per-call breakdown).
+    Every step is preceded by the L2 flush, outside the timed region."""
     graphs = capture_graphs(step)
-    names = list(graphs)
+    names = [nm for nm in graphs if nm != "step"]
     s = torch.cuda.current_stream()
     for _ in range(W):
         flush.zero_()
+        graphs["step"].replay()
         for nm in names:
             graphs[nm].replay()
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize()
+    for k in range(K):
+        flush.zero_()
+        evs[k][0].record(s)
+        graphs["step"].replay()
+        evs[k][1].record(s)
+    torch.cuda.synchronize()
+    barrier(world)
     for k in range(K):
         flush.zero_()
         ev[k][0].record(s)
@@ -336,8 +355,8 @@ def time_steps(step, K, W, world, flush):
             graphs[nm].replay()
             ev[k][j + 1].record(s)
     torch.cuda.synchronize()
-    barrier(world)
     times = {nm: [ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(K)] for j, nm in enumerate(names)}
+    times["step"] = [evs[k][0].elapsed_time(evs[k][1]) for k in range(K)]
     del graphs
     return times
 
@@ -512,8 +531,9 @@ def main():
     clk.start()
     times = time_steps(step, args.steps, args.warmup, world, flush)
     clocks = clk.stop()
-    per_step = [sum(ts) for ts in zip(*times.values())]
-    ms_step = max_over_ranks(statistics.fmean(per_step), world)
+    ms_step = max_over_ranks(statistics.fmean(times["step"]), world)
+    ms_calls = max_over_ranks(statistics.fmean([sum(ts) for ts in zip(*[times[nm] for nm in times if nm != "step"])]),
+                              world)
     ms_attn = max_over_ranks(statistics.fmean(times["attn"]), world)
     ms_acc = max_over_ranks(statistics.fmean(times["accept"]), world)
     ms_exp = max_over_ranks(statistics.fmean(times["expand"]), world) if "expand" in times else 0.0
@@ -566,6 +586,7 @@ def main():
                   "accept_gbs": round(step.accept_bytes / (ms_acc * 1e-3) / 1e9, 1),
                   "accept_nodes_per_s": step.B * step.T / (ms_acc * 1e-3)},
         "launches_per_step": step.launches_per_step(),
+        "ms_per_step_call_by_call": round(ms_calls, 5),
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": step.launches_per_step() * args.steps,

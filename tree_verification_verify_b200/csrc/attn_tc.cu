@@ -50,8 +50,9 @@ namespace tv {
 
 namespace tc {
 
-constexpr int kThreads = 256;
-constexpr int kWarpK = 4, kWarpMma = 5, kWarpV = 6, kWarpTree = 7;
+constexpr int kThreads = 384;
+constexpr int kSoftmaxThreads = 256;  // two threads per query row
+constexpr int kWarpK = 8, kWarpMma = 9, kWarpV = 10, kWarpTree = 11;
 constexpr int kRows = 128;          // M
 constexpr int kKeys = 128;          // keys per tile (N of QK, K of PV)
 constexpr int kD = 128;
@@ -97,6 +98,10 @@ struct Bars {
   int node_ok[kRows];               // root path of the tile's node is well formed
   uint64_t inbox_full;              // the cluster's copies into this CTA's inbox have landed
   alignas(16) float st_lse[kRows];  // this CTA's rows: log2-sum-exp (NaN: invalid)
+  uint64_t max_ready[2];            // both halves of every row have posted their tile maximum
+  uint64_t sum_ready;               // both halves have posted their row sums
+  float red_max[2][2][kRows];       // [tile parity][half][row] partial maxima
+  float red_l[2][kRows];            // [half][row] partial row sums
   alignas(16) float in_lse[kMaxInboxRows];  // merge inbox: log2-sum-exp of row (chunk, row)
 };
 
@@ -349,8 +354,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   const int nodes_here = min(kRows / G, n - i0);
   const bool has_tree = (chunk == C - 1);   // the last chunk is the shortest
   // this thread's query row (softmax warps)
-  const int row_node = i0 + tid / G;
-  const bool row_valid = tid < kRows && (tid / G) < nodes_here;
+  // softmax threads: query row tid % 128 (TMEM lane), column half tid / 128
+  const int row = tid & (kRows - 1);
+  const int half = tid >> 7;
+  const int row_node = i0 + row / G;
+  const bool row_valid = tid < kSoftmaxThreads && (row / G) < nodes_here;
   // rows [c * merge_per, (c + 1) * merge_per) of the tile are merged by CTA c
   const int merge_per = 4 * ((nodes_here * G + 4 * C - 1) / (4 * C));
 
@@ -367,7 +375,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < kKS; ++s) { mbar_init(&bars.k_full[s], 1); mbar_init(&bars.k_empty[s], 1); }
     for (int s = 0; s < kVS; ++s) { mbar_init(&bars.v_full[s], 1); mbar_init(&bars.v_empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&bars.s_full[s], 1); mbar_init(&bars.p_full[s], 4); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars.s_full[s], 1);
+      mbar_init(&bars.p_full[s], kSoftmaxThreads / 32);
+      mbar_init(&bars.max_ready[s], kSoftmaxThreads / 32);
+    }
+    mbar_init(&bars.sum_ready, kSoftmaxThreads / 32);
     mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.tree_info, 1);
     mbar_init(&bars.inbox_full, 1);
@@ -600,9 +613,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax warps 0-3
+    // ------------------------------------------------------------ softmax warps 0-7
+    // Row r is TMEM lane r: warps w and w + 4 share lanes 32 (w % 4) ..; warp
+    // w < 4 takes key columns 0-63 of every tile, warp w + 4 columns 64-127.
+    // The two halves exchange their tile maxima (shared memory + mbarrier),
+    // keep their own row sums, and add them at the end.
     const float sl2 = p.scale * 1.4426950408889634f;   // scores in log2 units
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t hcol = 64u * static_cast<uint32_t>(half);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     int ntot = nprefix, ntree = 0;
@@ -615,56 +633,59 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         if (!ok) break;
         ntree = (bars.nU + kKeys - 1) / kKeys;
         ntot += ntree;
-        my_ok = row_valid && bars.node_ok[tid / G] != 0;
+        my_ok = row_valid && bars.node_ok[row / G] != 0;
         cur = my_ok ? u_slot(bars, row_node) : -1;
         tree_known = true;
       }
       if (j >= ntot) break;
       const bool tree_tile = j >= nprefix;
       const int nk = tree_tile ? 0 : min(kKeys, k1 - (k0 + j * kKeys));
-      // key mask of the tile: four words, kept in registers
-      uint32_t mk0 = 0u, mk1 = 0u, mk2 = 0u, mk3 = 0u;
+      // key mask of this half's 64 columns: two words, kept in registers
+      uint32_t mkA = 0u, mkB = 0u;
       if (tree_tile) {
-        // ancestors of this row's node in slots [128 tt, 128 tt + 128); the
-        // tiles run downwards and slots decrease along the path, so the walk
-        // continues where the previous tile left it
+        // ancestors of this row's node in slots [128 tt + 64 half, + 64);
+        // the tiles run downwards and slots decrease along the path, so the
+        // walk continues where the previous tile left it
         const int lo = (ntree - 1 - (j - nprefix)) * kKeys;
         while (cur >= lo) {
-          if (cur < lo + kKeys) {
-            const int w = (cur - lo) >> 5;
+          const int w = (cur - lo) >> 5;           // 0..3 in the tile
+          if (cur < lo + kKeys && (w >> 1) == half) {
             const uint32_t bit = 1u << (cur & 31);
-            mk0 |= (w == 0) ? bit : 0u;
-            mk1 |= (w == 1) ? bit : 0u;
-            mk2 |= (w == 2) ? bit : 0u;
-            mk3 |= (w == 3) ? bit : 0u;
+            mkA |= (w & 1) == 0 ? bit : 0u;
+            mkB |= (w & 1) == 1 ? bit : 0u;
           }
           const uint16_t up = uparent[cur];
           cur = (up == kBadMark) ? -1 : static_cast<int>(up);
         }
       } else {
-        mk0 = nk >= 32 ? 0xffffffffu : ((1u << nk) - 1u);
-        mk1 = nk >= 64 ? 0xffffffffu : (nk <= 32 ? 0u : ((1u << (nk - 32)) - 1u));
-        mk2 = nk >= 96 ? 0xffffffffu : (nk <= 64 ? 0u : ((1u << (nk - 64)) - 1u));
-        mk3 = nk >= 128 ? 0xffffffffu : (nk <= 96 ? 0u : ((1u << (nk - 96)) - 1u));
+        const int nh = nk - 64 * half;              // valid keys in this half
+        mkA = nh >= 32 ? 0xffffffffu : (nh <= 0 ? 0u : ((1u << nh) - 1u));
+        mkB = nh >= 64 ? 0xffffffffu : (nh <= 32 ? 0u : ((1u << (nh - 32)) - 1u));
       }
       ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full[j & 1], (j >> 1) & 1, abort));
       if (!ok) break;
       fence_after();
-      float s[kKeys];
+      float s[64];
       const uint32_t scol = s_col(j);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(trow + scol + c * 32, s + c * 32);
+      tmem_ld32(trow + scol + hcol, s);
+      tmem_ld32(trow + scol + hcol + 32, s + 32);
       tmem_wait_ld();
-      // masked scores in log2 units; the maximum over four interleaved
-      // partial maxima (the maximum does not depend on the order)
+      // masked scores in log2 units; this half's maximum over four
+      // interleaved partial maxima (the maximum does not depend on order)
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < kKeys; ++c) {
-        const uint32_t mw = (c < 32) ? mk0 : (c < 64) ? mk1 : (c < 96) ? mk2 : mk3;
+      for (int c = 0; c < 64; ++c) {
+        const uint32_t mw = (c < 32) ? mkA : mkB;
         s[c] = ((mw >> (c & 31)) & 1u) ? s[c] * sl2 : -INFINITY;
         mx[c & 3] = fmaxf(mx[c & 3], s[c]);
       }
-      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float mh = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      bars.red_max[j & 1][half][row] = mh;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.max_ready[j & 1]);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars.max_ready[j & 1], (j >> 1) & 1, abort));
+      if (!ok) break;
+      const float mt = fmaxf(mh, bars.red_max[j & 1][half ^ 1][row]);
       const float m_new = fmaxf(m_run, mt);
       const bool first = (j == 0);
       const bool grow = !first && (m_new > m_run + 8.0f);
@@ -678,46 +699,47 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       const float mu = (m_run == -INFINITY) ? 0.f : m_run;
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kKeys; ++c) {
+      for (int c = 0; c < 64; ++c) {
         s[c] = ex2_approx(s[c] - mu);
         ps[c & 3] += s[c];
       }
       l_run = l_run * factor + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       if (__any_sync(0xffffffffu, grow)) {
         // O holds the tiles up to j - 1: wait for their P V, then rescale
+        // this half's 64 columns of O
         ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (j - 1) & 1, abort));
         if (!ok) break;
         fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           float o[32];
-          tmem_ld32(trow + kColO + c * 32, o);
+          tmem_ld32(trow + kColO + hcol + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= factor;
-          tmem_st32(trow + kColO + c * 32, o);
+          tmem_st32(trow + kColO + hcol + c * 32, o);
         }
       }
-      // P as bf16 pairs over the first 64 columns of the S buffer
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      // P as bf16 pairs over the first 64 columns of the S buffer: this
+      // half's keys 64 half .. 64 half + 63 are columns 32 half .. + 31
+      {
         uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(s[64 * h + 2 * e], s[64 * h + 2 * e + 1]);
-        tmem_st32u(trow + scol + 32 * h, pk);
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(s[2 * e], s[2 * e + 1]);
+        tmem_st32u(trow + scol + 32u * static_cast<uint32_t>(half), pk);
       }
       tmem_wait_st();
       if (!tree_tile && nk < kKeys) {
         // ragged prefix tile: V rows past the prefix end may hold anything
         ok = __all_sync(0xffffffffu, mbar_wait(&bars.v_full[j % kVS], (j / kVS) & 1, abort));
         if (!ok) break;
-        if (tid >= nk) {
+        if (half == 0 && row >= nk) {
           uint8_t* sv = gbase + kSmemV + (j % kVS) * kTileBytes;
           const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            *reinterpret_cast<uint4*>(sv + tid * 128 + c * 16) = z;
-            *reinterpret_cast<uint4*>(sv + kHalfBytes + tid * 128 + c * 16) = z;
+            *reinterpret_cast<uint4*>(sv + row * 128 + c * 16) = z;
+            *reinterpret_cast<uint4*>(sv + kHalfBytes + row * 128 + c * 16) = z;
           }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -733,28 +755,36 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     if (ok && ntot > 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (ntot - 2) & 1, abort));
     if (ok && ntot > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (ntot - 1) & 1, abort));
     fence_after();
-    const bool have = ok && l_run > 0.f;
-    const float inv = have ? 1.f / l_run : 0.f;
-    // this row's normalised O into the stage (the idle V ring; fp32,
-    // float4 q of row t at q ^ (t & 7)) and its log2-sum-exp
+    // the row sum is the two halves' sums
+    bars.red_l[half][row] = l_run;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.sum_ready);
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.sum_ready, 0, abort));
+    const float l_row = ok ? l_run + bars.red_l[half ^ 1][row] : 0.f;
+    const bool have = ok && l_row > 0.f;
+    const float inv = have ? 1.f / l_row : 0.f;
+    // this half of the row's normalised O into the stage (the idle V ring;
+    // fp32, float4 q of row t at q ^ (t & 7)) and the row's log2-sum-exp
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    float* stage = reinterpret_cast<float*>(gbase + kSmemStage) + tid * kD;
+    float* stage = reinterpret_cast<float*>(gbase + kSmemStage) + row * kD;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       float v[32];
-      tmem_ld32(trow + kColO + c * 32, v);
+      tmem_ld32(trow + kColO + hcol + c * 32, v);
       tmem_wait_ld();
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<float4*>(stage + (((c * 8 + q) ^ (tid & 7)) * 4)) =
+      for (int q = 0; q < 8; ++q) {
+        const int qq = 16 * half + c * 8 + q;
+        *reinterpret_cast<float4*>(stage + ((qq ^ (row & 7)) * 4)) =
             have ? make_float4(v[4 * q] * inv, v[4 * q + 1] * inv, v[4 * q + 2] * inv, v[4 * q + 3] * inv)
                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
     const bool good = !(has_tree && !my_ok) && !bad_len && ok;
-    bars.st_lse[tid] = !good ? NAN : (l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY);
+    if (half == 0) bars.st_lse[row] = !good ? NAN : (l_row > 0.f ? m_run + __log2f(l_row) : -INFINITY);
     // the stage is read by bulk copies (async proxy)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    if (row_valid && has_tree && !my_ok) set_status(p.status, TV_DEV_BAD_PARENT);
+    if (half == 0 && row_valid && has_tree && !my_ok) set_status(p.status, TV_DEV_BAD_PARENT);
     if (bad_len && has_tree && tid == 0) set_status(p.status, TV_DEV_BAD_LEN);
   }
 
