@@ -71,7 +71,9 @@ SHAPES = [
     (2, 70, 16, 2, 128, [0, 700], "bf16", "recursive"),
     (1, 300, 32, 8, 128, [200], "bf16", "chain"),        # deep: 3 gathered tree tiles
     (2, 129, 8, 1, 128, [333, 1], "bf16", "binary"),
-    (1, 600, 64, 8, 128, [5000], "bf16", "recursive"),   # split prefix + fused merge
+    (1, 600, 64, 8, 128, [5000], "bf16", "recursive"),   # split prefix + cluster merge
+    (1, 300, 32, 8, 128, [2000], "bf16", "chain"),       # ragged last row tile after 3 tree tiles
+    (1, 1000, 64, 8, 128, [300], "bf16", "chain"),       # 8 tree tiles per row tile
 ]
 
 
@@ -191,6 +193,21 @@ def test_sparse_small_offsets():
                      offset_frac=0.1, block_size=bs, sparse_topk=8)
     rows = {(b, i) for b in range(2) for i in range(T)}
     _check_sparse(case, rows, 2, T, 2, 4, 8)
+
+
+@pytest.mark.parametrize("Hq,Hkv,d,dtype,bs,k", [
+    (8, 8, 64, "bf16", 100, 6),     # G = 1, blocks wider than one 64-key tile, ragged last block
+    (32, 4, 128, "bf16", 16, 12),   # G = 8, narrow blocks
+    (64, 2, 32, "fp32", 40, 5),     # G = 32 (two heads per warp), fp32, d = 32
+])
+def test_sparse_shapes(Hq, Hkv, d, dtype, bs, k):
+    """The block top-k path over head groups, head dims, dtypes and block
+    widths (blocks of more than 64 keys are streamed in two tiles)."""
+    T, L = 11, [bs * 9 + 7, bs * 3]
+    case = attn_case(2, T, Hq, Hkv, d, L, dtype, tree_random_recursive(T, torch.Generator().manual_seed(2)),
+                     seed=9, offset_frac=0.2, block_size=bs, sparse_topk=k)
+    rows = {(b, i) for b in range(2) for i in range(T)}
+    _check_sparse(case, rows, 2, T, Hkv, Hq // Hkv, k)
 
 
 def test_full_size_sparse_sampled():
