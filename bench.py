@@ -569,6 +569,8 @@ def main():
                     "peak": bf16, "unit": "TFLOP/s", "frac": round(achieved / bf16, 4), "traffic": None,
                     "peak_source": src, "algorithmic_flops": step.attn_flops}
             tk = "attn_tc_kernel"
+    if tk == "attn_tc_kernel" and step.attn_path == 1:
+        roof["kernel"] = "attn_tc_kernel (tree_verify_attn: one launch)"
     if step.attn_path != 1 and tk == "attn_tc_kernel":
         roof["kernel"] = "tree_verify_attn (all launches)"
     else:
