@@ -9,7 +9,7 @@ tree tokens per second per layer over all ranks.  Inputs are synthetic
 (seeded Gaussian activations and logits of those shapes).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--config llama3_8b|specexec70b|serving|longctx|longctx_sparse]
+                    [--config llama3_8b|specexec70b|serving|longctx|longctx_sparse|tiny]
 
 Timing: the step's calls are captured once into one CUDA graph (and each
 call into a graph of its own); W untimed warm-up steps, then K steps of the
@@ -511,7 +511,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="llama3_8b",
-                    choices=["llama3_8b", "specexec70b", "serving", "longctx", "longctx_sparse"])
+                    choices=["llama3_8b", "specexec70b", "serving", "longctx", "longctx_sparse", "tiny"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
