@@ -294,14 +294,18 @@ TV_API tv_status tree_expand_topb(const tv_expand_args* a, void* ws, size_t ws_b
  * ---------------------------------------------------------------------- */
 /* Which kernels tree_verify_attn would run for these arguments:
  * 0 = CUDA-core split-KV, 1 = tcgen05 tensor-core prefix kernel,
- * 2 = block top-k sparse path, -1 = the arguments are rejected. */
+ * 2 = block top-k sparse path on CUDA cores, 3 = block top-k sparse path on
+ * the tensor-core kernel (bf16, d = 128, blocks of 64, G >= 4),
+ * -1 = the arguments are rejected. */
 TV_API int32_t tv_attn_path(const tv_attn_args* a);
 /* How many kernels tree_verify_attn launches for these arguments (0 when
  * B or T is 0, -1 when the arguments are rejected): 1 for the tensor-core
  * kernel (its prefix chunks are merged inside the launch), 3 on the
  * CUDA-core path (prefix, tree paths, merge), 5 or 6 on
- * the block top-k path (block means unless the caller passes them, block
- * scores, block selection, sparse prefix, tree paths, merge).  Host only; nothing runs. */
+ * the block top-k CUDA-core path (block means unless the caller passes
+ * them, block scores, block selection, sparse prefix, tree paths, merge),
+ * 3 or 4 on the block top-k tensor-core path (block means, scores,
+ * selection, the tensor-core kernel).  Host only; nothing runs. */
 TV_API int32_t tv_attn_launches(const tv_attn_args* a);
 /* Library version, e.g. "treeverify 0.1.0 sm_100a". */
 TV_API const char* tree_verify_version(void);

@@ -193,6 +193,8 @@ def test_sparse_small_offsets():
                      offset_frac=0.1, block_size=bs, sparse_topk=8)
     rows = {(b, i) for b in range(2) for i in range(T)}
     _check_sparse(case, rows, 2, T, 2, 4, 8)
+    import tree_verification_verify_b200 as tv
+    assert tv.last_attn_path == 3          # bf16, d = 128, blocks of 64, G = 4: tensor cores
 
 
 @pytest.mark.parametrize("Hq,Hkv,d,dtype,bs,k", [
@@ -208,6 +210,8 @@ def test_sparse_shapes(Hq, Hkv, d, dtype, bs, k):
                      seed=9, offset_frac=0.2, block_size=bs, sparse_topk=k)
     rows = {(b, i) for b in range(2) for i in range(T)}
     _check_sparse(case, rows, 2, T, Hkv, Hq // Hkv, k)
+    import tree_verification_verify_b200 as tv
+    assert tv.last_attn_path == 2          # outside the tensor-core variant: CUDA cores
 
 
 def test_full_size_sparse_sampled():
@@ -216,3 +220,5 @@ def test_full_size_sparse_sampled():
     rows = _sample_rows(c["B"], c["T"], 3, 2)
     checked, near, st = _check_sparse(case, rows, c["B"], c["T"], c["Hkv"], c["Hq"] // c["Hkv"], 32)
     assert st == 0
+    import tree_verification_verify_b200 as tv
+    assert tv.last_attn_path == 3

@@ -239,7 +239,8 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent, n_
 # Which attention kernels the last tree_verify_attn call ran (tv_attn_path).
 last_attn_path = None
 last_attn_launches = None
-ATTN_PATHS = {0: "cuda-core split-KV", 1: "tcgen05 prefix", 2: "block top-k sparse"}
+ATTN_PATHS = {0: "cuda-core split-KV", 1: "tcgen05 prefix", 2: "block top-k sparse (cuda cores)",
+              3: "block top-k sparse (tcgen05)"}
 
 
 # --------------------------------------------------------------- acceptance

@@ -24,6 +24,7 @@ struct AttnParams {
   const float* kbar;           // [B][nblk_max][Hkv][d] (caller's or workspace)
   int32_t* sel;                // [B][T][Hkv][topk] kept blocks (workspace)
   float* scores;               // [B][T][Hkv][nblk_max] cheap block scores (workspace)
+  int tc_sparse;               // the tensor-core kernel runs the block top-k variant
   int32_t* sel_out;            // caller's copy or NULL
   // split-KV plan and workspace
   int nchunk;                  // prefix chunks (the tree part is chunk nchunk)

@@ -58,7 +58,11 @@ constexpr int kKeys = 128;          // keys per tile (N of QK, K of PV)
 constexpr int kD = 128;
 constexpr int kKS = 3;              // K ring stages
 constexpr int kVS = 2;              // V ring stages
-constexpr int kMaxT = 4096;         // tree nodes handled by this kernel
+constexpr int kMaxT = 2048;         // tree nodes handled by this kernel
+constexpr int kMaxUnion = 1024;     // block top-k: kept blocks in the union of a row tile
+constexpr int kMaxTopk = 64;        // block top-k: kept blocks per (node, kv head)
+constexpr int kMaxSpNodes = 32;     // block top-k: nodes per row tile (G >= 4)
+constexpr int kMaxBlk = 4096;       // block top-k: 64-key prefix blocks
 constexpr int kMaxCluster = 8;      // chunks per row tile
 constexpr uint32_t kHalfBytes = kRows * 128;            // 128 rows x 128 B
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;         // 32 KB (d = 128 bf16)
@@ -68,7 +72,10 @@ constexpr uint32_t kSmemV = kSmemK + kKS * kTileBytes;
 constexpr uint32_t kSmemPar = kSmemV + kVS * kTileBytes;  // parent[] (u16)
 constexpr uint32_t kSmemUL = kSmemPar + kMaxT * 2;        // U: slot -> node (u16)
 constexpr uint32_t kSmemUP = kSmemUL + kMaxT * 2;         // U: slot -> parent's slot (u16)
-constexpr uint32_t kSmemBytes = kSmemUP + kMaxT * 2;      // 216 KB
+constexpr uint32_t kSmemUB = kSmemUP + kMaxT * 2;         // block top-k: union blocks (u16)
+constexpr uint32_t kSmemNL = kSmemUB + kMaxUnion * 2;     // block top-k: kept lists per node (u16)
+constexpr uint32_t kSmemUBM = kSmemNL + kMaxSpNodes * kMaxTopk * 2;   // block top-k: union bitmap
+constexpr uint32_t kSmemBytes = kSmemUBM + kMaxBlk / 8;   // 211 KB
 constexpr uint32_t kSmemInbox = kSmemK;                   // merge: fp32 O rows copied in by the cluster
 constexpr uint32_t kSmemStage = kSmemV;                   // merge: this CTA's fp32 O rows (idle V ring)
 constexpr int kMaxInboxRows = 144;                        // max over C of C * per (per = 4 * ceil(128 / 4C))
@@ -90,9 +97,11 @@ struct Bars {
   uint64_t s_full[2], p_full[2];
   uint64_t pv_done;
   uint64_t tree_info;
+  uint64_t sparse_info;             // block top-k: the union of kept blocks is listed
   uint32_t tmem_base;
   int abort;
   int nU;                           // nodes in the union of root paths
+  int nUB;                          // block top-k: blocks in the union of the tile's kept blocks
   uint32_t bm[kMaxT / 32];          // node bitmap of U
   int pre[kMaxT / 32];              // marked nodes below each bitmap word
   int node_ok[kRows];               // root path of the tile's node is well formed
@@ -324,9 +333,15 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* b, uint32_t parity) 
 
 using namespace tc;
 
+// SPARSE: block top-k verification attention.  The prefix tiles are then the
+// union of the 64-key blocks that the tile's nodes keep (two blocks per key
+// tile, loaded with 64-key boxes tmap_k64 / tmap_v64), and a row keeps a
+// block only when its node selected it; one chunk per row tile.
+template <bool SPARSE>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-               const __grid_constant__ CUtensorMap tmap_v, AttnParams p) {
+               const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_k64,
+               const __grid_constant__ CUtensorMap tmap_v64, AttnParams p) {
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ Bars bars;
   cg::cluster_group cl = cg::this_cluster();
@@ -350,7 +365,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   const int L = bad_len ? 0 : Lraw;
   const int k0 = chunk * p.chunk_len;
   const int k1 = min(k0 + p.chunk_len, L);
-  const int nprefix = (k1 > k0) ? (k1 - k0 + kKeys - 1) / kKeys : 0;
+  // key tiles of the prefix: known here (dense), or once the union of the
+  // kept blocks is listed (block top-k)
+  int nprefix = SPARSE ? 0 : ((k1 > k0) ? (k1 - k0 + kKeys - 1) / kKeys : 0);
   const int nodes_here = min(kRows / G, n - i0);
   const bool has_tree = (chunk == C - 1);   // the last chunk is the shortest
   // this thread's query row (softmax warps)
@@ -369,7 +386,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   uint16_t* spar = reinterpret_cast<uint16_t*>(gbase + kSmemPar);
   uint16_t* ulist = reinterpret_cast<uint16_t*>(gbase + kSmemUL);
   uint16_t* uparent = reinterpret_cast<uint16_t*>(gbase + kSmemUP);
+  uint16_t* ublk = reinterpret_cast<uint16_t*>(gbase + kSmemUB);
+  uint16_t* nlist = reinterpret_cast<uint16_t*>(gbase + kSmemNL);
+  uint32_t* ubm = reinterpret_cast<uint32_t*>(gbase + kSmemUBM);
   volatile int* abort = &bars.abort;
+  // block top-k: blocks 2 jt and 2 jt + 1 of the union form key tile jt
+  auto blk_of = [&](int slot) -> int { return slot < bars.nUB ? static_cast<int>(ublk[slot]) : -1; };
+  auto blk_keys = [&](int blk) -> int { return blk < 0 ? 0 : min(64, L - 64 * blk); };
 
   if (tid == 0) {
     mbar_init(&bars.q_full, 1);
@@ -383,9 +406,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     mbar_init(&bars.sum_ready, kSoftmaxThreads / 32);
     mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.tree_info, 1);
+    mbar_init(&bars.sparse_info, 1);
     mbar_init(&bars.inbox_full, 1);
     bars.abort = 0;
     bars.nU = 0;
+    bars.nUB = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     // the bytes the cluster will copy into this CTA's inbox
@@ -406,6 +431,46 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
 
   if (warp == kWarpTree) {
     // ------------------------------------------------------------ tree bookkeeping
+    if (SPARSE) {
+      // the kept blocks of every node of the tile (ascending, 0xFFFF past
+      // the end) and their union, listed in ascending block order
+      const int nblk = (L + 63) / 64;
+      const int nbw = (nblk + 31) >> 5;
+      for (int w = lane; w < nbw; w += 32) ubm[w] = 0u;
+      __syncwarp();
+      const int32_t* sel = p.sel + (static_cast<int64_t>(b) * p.T + i0) * p.Hkv * p.topk + g * p.topk;
+      for (int e = lane; e < nodes_here * p.topk; e += 32) {
+        const int r = e / p.topk, t = e % p.topk;
+        const int j = sel[static_cast<int64_t>(r) * p.Hkv * p.topk + t];
+        const bool kept = j >= 0 && j < nblk;
+        nlist[r * kMaxTopk + t] = kept ? static_cast<uint16_t>(j) : 0xFFFFu;
+        if (kept) atomicOr(&ubm[j >> 5], 1u << (j & 31));
+      }
+      __syncwarp();
+      const int per = (nbw + 31) / 32;
+      const int lo = min(lane * per, nbw), hi = min(lo + per, nbw);
+      int cnt = 0;
+      for (int w = lo; w < hi; ++w) cnt += __popc(ubm[w]);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int run = incl - cnt;
+      for (int w = lo; w < hi; ++w) {
+        uint32_t m = ubm[w];
+        while (m) {
+          const int bit = __ffs(m) - 1;
+          ublk[run++] = static_cast<uint16_t>(w * 32 + bit);
+          m &= m - 1u;
+        }
+      }
+      const int nUB = __shfl_sync(0xffffffffu, incl, 31);
+      if (lane == 0) bars.nUB = nUB;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.sparse_info);
+    }
     if (has_tree) {
       for (int j = lane; j < n; j += 32) {
         const int pj = par[j];
@@ -477,10 +542,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       tma_load_4d(&tmap_q, sq, &bars.q_full, 0, g * G, i0, b);
       tma_load_4d(&tmap_q, sq + kHalfBytes, &bars.q_full, 64, g * G, i0, b);
     }
+    bool sparse_ok = true;
+    if (SPARSE) {
+      bool w = true;
+      if (lane == 0) w = mbar_wait(&bars.sparse_info, 0, abort);
+      sparse_ok = __all_sync(0xffffffffu, w);
+      nprefix = sparse_ok ? (bars.nUB + 1) / 2 : 0;
+    }
     int ntot = nprefix, ntree = 0;
     bool tree_known = !has_tree;
     int issued = 0;
-    for (int j = 0;; ++j) {
+    for (int j = 0; sparse_ok; ++j) {
       if (!tree_known && j == nprefix) {
         bool w = true;
         if (lane == 0) w = mbar_wait(&bars.tree_info, 0, abort);
@@ -497,7 +569,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         if (!__all_sync(0xffffffffu, w)) break;
       }
       const uint32_t dst = ring + s * kTileBytes;
-      if (j < nprefix) {
+      if (SPARSE && j < nprefix) {
+        // kept blocks 2 j and 2 j + 1 of the union, 64 keys each, as rows
+        // 0-63 and 64-127 of the tile
+        if (lane == 0) {
+          const CUtensorMap* map64 = isk ? &tmap_k64 : &tmap_v64;
+          const int ja = blk_of(2 * j), jb = blk_of(2 * j + 1);
+          mbar_expect_tx(&full[s], (jb >= 0 ? 2u : 1u) * (kTileBytes / 2));
+          tma_load_4d(map64, dst, &full[s], 0, g, 64 * ja, b);
+          tma_load_4d(map64, dst + kHalfBytes, &full[s], 64, g, 64 * ja, b);
+          if (jb >= 0) {
+            tma_load_4d(map64, dst + 64 * 128, &full[s], 0, g, 64 * jb, b);
+            tma_load_4d(map64, dst + kHalfBytes + 64 * 128, &full[s], 64, g, 64 * jb, b);
+          }
+        }
+      } else if (j < nprefix) {
         if (lane == 0) {
           const int kb = k0 + j * kKeys;
           mbar_expect_tx(&full[s], kTileBytes);
@@ -537,9 +623,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      bool ok = true;
+      if (SPARSE) {
+        ok = mbar_wait(&bars.sparse_info, 0, abort);
+        nprefix = ok ? (bars.nUB + 1) / 2 : 0;
+      }
       int ntot = nprefix;
       bool tree_known = !has_tree;
-      bool ok = true;
       // the tree tiles follow the prefix tiles; their count is known once
       // the tree warp has built U
       auto know = [&](int upto) -> bool {
@@ -566,7 +656,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         mma_commit(&bars.s_full[j & 1]);
         ++s_issued;
       };
-      ok = know(0);
+      ok = ok && know(0);
       if (ok && ntot > 0) ok = mbar_wait(&bars.q_full, 0, abort);
       for (int j = 0; j < 2 && ok; ++j) {
         ok = know(j);
@@ -623,10 +713,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     const uint32_t hcol = 64u * static_cast<uint32_t>(half);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
+    if (SPARSE) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars.sparse_info, 0, abort));
+      nprefix = ok ? (bars.nUB + 1) / 2 : 0;
+    }
     int ntot = nprefix, ntree = 0;
     bool my_ok = true;
     bool tree_known = !has_tree;
     int cur = -1;                 // walk position (slot) on this row's root path
+    int lcur = 0;                 // block top-k: cursor into this row's node's kept list
+    const uint16_t* mylist = nlist + (row / G) * kMaxTopk;
     for (int j = 0; ok; ++j) {
       if (!tree_known && j == nprefix) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bars.tree_info, 0, abort));
@@ -639,7 +735,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       }
       if (j >= ntot) break;
       const bool tree_tile = j >= nprefix;
-      const int nk = tree_tile ? 0 : min(kKeys, k1 - (k0 + j * kKeys));
+      const int nk = (tree_tile || SPARSE) ? 0 : min(kKeys, k1 - (k0 + j * kKeys));
       // key mask of this half's 64 columns: two words, kept in registers
       uint32_t mkA = 0u, mkB = 0u;
       if (tree_tile) {
@@ -657,6 +753,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           const uint16_t up = uparent[cur];
           cur = (up == kBadMark) ? -1 : static_cast<int>(up);
         }
+      } else if (SPARSE) {
+        // this half's block (slot 2 j + half of the union): kept by this
+        // row's node?  Both the kept list and the union ascend, so the
+        // cursor only moves forward.
+        const int blk = blk_of(2 * j + half);
+        bool member = false;
+        if (row_valid && blk >= 0) {
+          while (lcur < p.topk && mylist[lcur] < blk) ++lcur;
+          member = lcur < p.topk && mylist[lcur] == blk;
+        }
+        const int nh = member ? blk_keys(blk) : 0;
+        mkA = nh >= 32 ? 0xffffffffu : (nh <= 0 ? 0u : ((1u << nh) - 1u));
+        mkB = nh >= 64 ? 0xffffffffu : (nh <= 32 ? 0u : ((1u << (nh - 32)) - 1u));
       } else {
         const int nh = nk - 64 * half;              // valid keys in this half
         mkA = nh >= 32 ? 0xffffffffu : (nh <= 0 ? 0u : ((1u << nh) - 1u));
@@ -729,11 +838,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         tmem_st32u(trow + scol + 32u * static_cast<uint32_t>(half), pk);
       }
       tmem_wait_st();
-      if (!tree_tile && nk < kKeys) {
-        // ragged prefix tile: V rows past the prefix end may hold anything
+      // V rows that are not keys of this tile (past the prefix end, or an
+      // absent second block) may hold anything: zero them
+      int vka = 64, vkb = 64;
+      if (SPARSE && !tree_tile) { vka = blk_keys(blk_of(2 * j)); vkb = blk_keys(blk_of(2 * j + 1)); }
+      const bool ragged = SPARSE ? (!tree_tile && (vka < 64 || vkb < 64)) : (!tree_tile && nk < kKeys);
+      if (ragged) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bars.v_full[j % kVS], (j / kVS) & 1, abort));
         if (!ok) break;
-        if (half == 0 && row >= nk) {
+        const bool dead_row = SPARSE ? (row < 64 ? row >= vka : row - 64 >= vkb) : row >= nk;
+        if (half == 0 && dead_row) {
           uint8_t* sv = gbase + kSmemV + (j % kVS) * kTileBytes;
           const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
@@ -936,6 +1050,18 @@ bool attn_tc_supported(const tv_attn_args* a) {
   return major == 10 && minor == 0;
 }
 
+bool attn_tc_sparse_supported(const tv_attn_args* a) {
+  if (a->sparse_topk <= 0 || a->block_size != 64 || a->sparse_topk > kMaxTopk) return false;
+  if (a->Hq % a->Hkv != 0) return false;
+  const int G = a->Hq / a->Hkv;
+  if (G < 4 || 128 % G != 0) return false;                  // at most 32 nodes per row tile
+  if ((kRows / G) * a->sparse_topk > kMaxUnion) return false;
+  if ((a->Lmax + 63) / 64 > kMaxBlk) return false;
+  tv_attn_args dense = *a;
+  dense.sparse_topk = 0;
+  return attn_tc_supported(&dense);
+}
+
 int attn_tc_active_clusters(int c) {
   // clusters of c chunk CTAs that can be resident at once (cached per device)
   static int cached[64][kMaxCluster + 1];
@@ -946,7 +1072,7 @@ int attn_tc_active_clusters(int c) {
   if (done[dev][c]) return cached[dev][c];
   int n = 0;
   const size_t smem = kSmemBytes + 1024;
-  if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(c, 1, 1);
@@ -959,7 +1085,7 @@ int attn_tc_active_clusters(int c) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel<false>, &cfg) != cudaSuccess) n = 0;
   }
   cudaGetLastError();
   cached[dev][c] = n;
@@ -968,16 +1094,25 @@ int attn_tc_active_clusters(int c) {
 }
 
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream) {
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mk64, mv64;
   const int G = p.G;
   if (p.nchunk < 1 || p.nchunk > kMaxCluster) return cudaErrorInvalidValue;
+  if (p.tc_sparse && p.nchunk != 1) return cudaErrorInvalidValue;
   if (!make_map(&mq, p.q, p.d, p.Hq, p.T, p.B, p.q_sh, p.q_st, p.q_sb, G, kRows / G) ||
       !make_map(&mk, p.kc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, kKeys) ||
       !make_map(&mv, p.vc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, kKeys))
     return cudaErrorInvalidValue;
+  if (p.tc_sparse) {
+    if (!make_map(&mk64, p.kc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, 64) ||
+        !make_map(&mv64, p.vc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, 64))
+      return cudaErrorInvalidValue;
+  } else {
+    mk64 = mk;
+    mv64 = mv;
+  }
+  auto kernel = p.tc_sparse ? attn_tc_kernel<true> : attn_tc_kernel<false>;
   const size_t smem = kSmemBytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int ntiles = (p.T + p.node_tile - 1) / p.node_tile;
   cudaLaunchConfig_t cfg = {};
@@ -992,7 +1127,7 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, mq, mk, mv, p);
+  e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, mk64, mv64, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

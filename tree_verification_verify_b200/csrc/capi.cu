@@ -16,6 +16,7 @@ cudaError_t launch_expand(const tv_expand_args* a, cudaStream_t stream);
 bool attn_tc_supported(const tv_attn_args* a);
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream);
 int attn_tc_active_clusters(int c);
+bool attn_tc_sparse_supported(const tv_attn_args* a);
 cudaError_t launch_block_means(const AttnParams& p, float* kbar, cudaStream_t stream);
 cudaError_t launch_block_select(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attn_sparse(const AttnParams& p, cudaStream_t stream);
@@ -40,6 +41,7 @@ bool ws_ok(const void* ws, size_t ws_bytes, size_t need) {
 struct AttnPlan {
   bool tc;            // tensor-core prefix kernel
   bool sparse;
+  bool tc_sparse;     // block top-k on the tensor-core kernel
   int nchunk, chunk_len, node_tile, nblk_max;
   size_t off_o, off_lse, off_ok, off_kbar, off_sel, off_scores, total;
 };
@@ -68,8 +70,9 @@ AttnPlan plan_attn(const tv_attn_args* a) {
   const int G = a->Hq / a->Hkv;
   pl.sparse = a->sparse_topk > 0;
   pl.tc = !pl.sparse && attn_tc_supported(a);
+  pl.tc_sparse = pl.sparse && attn_tc_sparse_supported(a);
   pl.node_tile = G >= 64 ? 1 : 64 / G;
-  if (pl.tc) pl.node_tile = 128 / G > 0 ? 128 / G : 1;
+  if (pl.tc || pl.tc_sparse) pl.node_tile = 128 / G > 0 ? 128 / G : 1;
   const int64_t ntiles = (a->T + pl.node_tile - 1) / pl.node_tile;
   const int64_t units = static_cast<int64_t>(a->B) * a->Hkv * (ntiles > 0 ? ntiles : 1);
   if (a->Lmax == 0 || pl.sparse) {
@@ -117,7 +120,7 @@ AttnPlan plan_attn(const tv_attn_args* a) {
   const size_t rows = static_cast<size_t>(a->B) * a->T * a->Hq;
   // the tensor-core path merges its chunks on chip; the other paths merge
   // partials (prefix chunks + the tree-path partial) through the workspace
-  const size_t nparts = pl.tc ? 0 : static_cast<size_t>(pl.nchunk) + 1;
+  const size_t nparts = (pl.tc || pl.tc_sparse) ? 0 : static_cast<size_t>(pl.nchunk) + 1;
   size_t off = kTicketBytes;
   pl.off_o = off;  off = align256(off + nparts * rows * a->d * sizeof(float));
   pl.off_lse = off; off = align256(off + nparts * rows * sizeof(float));
@@ -148,14 +151,14 @@ extern "C" size_t tree_verify_attn_workspace_size(const tv_attn_args* a) {
 extern "C" int32_t tv_attn_path(const tv_attn_args* a) {
   if (check_attn(a) != TV_OK) return -1;
   const AttnPlan pl = plan_attn(a);
-  return pl.sparse ? 2 : (pl.tc ? 1 : 0);
+  return pl.sparse ? (pl.tc_sparse ? 3 : 2) : (pl.tc ? 1 : 0);
 }
 
 extern "C" int32_t tv_attn_launches(const tv_attn_args* a) {
   if (check_attn(a) != TV_OK) return -1;
   if (a->B == 0 || a->T == 0) return 0;
   const AttnPlan pl = plan_attn(a);
-  if (pl.sparse) return (a->k_block_mean ? 0 : 1) + 5;
+  if (pl.sparse) return (a->k_block_mean ? 0 : 1) + 2 + (pl.tc_sparse ? 1 : 3);
   if (pl.tc) return 1;
   return 3;
 }
@@ -202,6 +205,11 @@ extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws
     }
     e = launch_block_select(p, s);
     if (e != cudaSuccess) return from_cuda(e);
+    if (pl.tc_sparse) {
+      // the kept blocks' union as key tiles of the tensor-core kernel
+      p.tc_sparse = 1;
+      return from_cuda(launch_attn_tc(p, s));
+    }
     e = launch_attn_sparse(p, s);
   } else if (pl.tc) {
     // one kernel: prefix tiles, tree tiles and the cluster merge of the chunks
