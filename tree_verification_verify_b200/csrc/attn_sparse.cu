@@ -57,16 +57,29 @@ __global__ void __launch_bounds__(256) block_means_kernel(AttnParams p, float* k
 #pragma unroll
   for (int x = 0; x < E; ++x) acc[x] = 0.f;
   if (kg < groups) {
-    for (int t = lo + kg; t < hi; t += groups) {
-      const int64_t off = b * p.kv_sb + static_cast<int64_t>(t) * p.kv_sl + g * p.kv_sh + c * E;
-      if (vec) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(kc + off));
-        const T* ev = reinterpret_cast<const T*>(&raw);
+    // four keys' loads in flight per batch (added in key order)
+    for (int t0 = lo + kg; t0 < hi; t0 += 4 * groups) {
+      uint4 raw[4];
 #pragma unroll
-        for (int x = 0; x < E; ++x) acc[x] += to_f32(ev[x]);
-      } else {
+      for (int u = 0; u < 4; ++u) {
+        const int t = t0 + u * groups;
+        const int64_t off = b * p.kv_sb + static_cast<int64_t>(t) * p.kv_sl + g * p.kv_sh + c * E;
+        if (t < hi && vec) raw[u] = __ldg(reinterpret_cast<const uint4*>(kc + off));
+        else raw[u] = make_uint4(0u, 0u, 0u, 0u);
+      }
 #pragma unroll
-        for (int x = 0; x < E; ++x) acc[x] += to_f32(kc[off + x]);
+      for (int u = 0; u < 4; ++u) {
+        const int t = t0 + u * groups;
+        if (t >= hi) break;
+        if (vec) {
+          const T* ev = reinterpret_cast<const T*>(&raw[u]);
+#pragma unroll
+          for (int x = 0; x < E; ++x) acc[x] += to_f32(ev[x]);
+        } else {
+          const int64_t off = b * p.kv_sb + static_cast<int64_t>(t) * p.kv_sl + g * p.kv_sh + c * E;
+#pragma unroll
+          for (int x = 0; x < E; ++x) acc[x] += to_f32(kc[off + x]);
+        }
       }
     }
   }
@@ -87,12 +100,13 @@ __global__ void __launch_bounds__(256) block_means_kernel(AttnParams p, float* k
 // thread, operands d-major in shared memory).  Each score is one fp32 dot
 // product over d in order.
 constexpr int kScTile = 64;
+constexpr int kScPad = kScTile + 4;        // row stride of the d-major operands (fewer bank conflicts)
 
 template <typename T>
 __global__ void __launch_bounds__(256) block_scores_kernel(AttnParams p) {
-  extern __shared__ float scs[];                     // Qs[d][64], Ks[d][64]
+  extern __shared__ float scs[];                     // Qs[d][kScPad], Ks[d][kScPad]
   float* Qs = scs;
-  float* Ks = scs + p.d * kScTile;
+  float* Ks = scs + p.d * kScPad;
   const int j0 = blockIdx.x * kScTile;
   const int b = blockIdx.y / p.Hkv, g = blockIdx.y % p.Hkv;
   const int i0 = blockIdx.z * kScTile;
@@ -103,7 +117,7 @@ __global__ void __launch_bounds__(256) block_scores_kernel(AttnParams p) {
                     ((p.q_sb | p.q_st | p.q_sh) * static_cast<int64_t>(sizeof(T))) % 16 == 0;
   const int nch = p.d / E;
   for (int e = tid; e < kScTile * nch; e += blockDim.x) {
-    const int r = e / nch, c = e % nch;
+    const int r = e % kScTile, c = e / kScTile;     // consecutive threads: consecutive rows
     float qsum[E];
 #pragma unroll
     for (int x = 0; x < E; ++x) qsum[x] = 0.f;
@@ -121,13 +135,13 @@ __global__ void __launch_bounds__(256) block_scores_kernel(AttnParams p) {
         }
       }
 #pragma unroll
-    for (int x = 0; x < E; ++x) Qs[(c * E + x) * kScTile + r] = qsum[x];
+    for (int x = 0; x < E; ++x) Qs[(c * E + x) * kScPad + r] = qsum[x];
   }
   for (int e = tid; e < kScTile * p.d; e += blockDim.x) {
     const int r = e / p.d, dd = e % p.d;
     float kb = 0.f;
     if (j0 + r < p.nblk_max) kb = p.kbar[((static_cast<int64_t>(b) * p.nblk_max + j0 + r) * p.Hkv + g) * p.d + dd];
-    Ks[dd * kScTile + r] = kb;
+    Ks[dd * kScPad + r] = kb;
   }
   __syncthreads();
   const int ty = tid >> 4, tx = tid & 15;
@@ -137,8 +151,8 @@ __global__ void __launch_bounds__(256) block_scores_kernel(AttnParams p) {
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
   for (int dd = 0; dd < p.d; ++dd) {
-    const float4 qa = *reinterpret_cast<const float4*>(Qs + dd * kScTile + ty * 4);
-    const float4 kb = *reinterpret_cast<const float4*>(Ks + dd * kScTile + tx * 4);
+    const float4 qa = *reinterpret_cast<const float4*>(Qs + dd * kScPad + ty * 4);
+    const float4 kb = *reinterpret_cast<const float4*>(Ks + dd * kScPad + tx * 4);
     const float qv[4] = {qa.x, qa.y, qa.z, qa.w}, kv[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
     for (int a = 0; a < 4; ++a)
@@ -438,7 +452,7 @@ cudaError_t launch_block_means(const AttnParams& p, float* kbar, cudaStream_t s)
 cudaError_t launch_block_select(const AttnParams& p, cudaStream_t s) {
   cudaError_t e;
   if (p.nblk_max > 0) {
-    const size_t ssm = 2 * sizeof(float) * static_cast<size_t>(p.d) * kScTile;
+    const size_t ssm = 2 * sizeof(float) * static_cast<size_t>(p.d) * kScPad;
     dim3 sgrid((p.nblk_max + kScTile - 1) / kScTile, p.B * p.Hkv, (p.T + kScTile - 1) / kScTile);
     if (p.dtype == TV_BF16) {
       e = cudaFuncSetAttribute(block_scores_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
