@@ -114,16 +114,6 @@ __device__ __forceinline__ double warp_incl_scan(double v) {
   return v;
 }
 
-// exp(a) for a float64 argument a <= 0, from the single-precision expf of
-// the rounded argument times a first-order correction for the rounding
-// residual: exp(hi + lo) = exp(hi) * (1 + lo + ...), |lo| <= 2^-24 |a|.
-__device__ __forceinline__ double exp_neg(double a) {
-  if (!(a > -200.0)) return 0.0;
-  const float hi = static_cast<float>(a);
-  const double lo = a - static_cast<double>(hi);
-  return static_cast<double>(expf(hi)) * (1.0 + lo);
-}
-
 // ---------------------------------------------------------------- loads
 
 // Four consecutive fp32 values starting at element e of a row of n values;
