@@ -249,6 +249,7 @@ struct SegStream {
   uint64_t* bar;        // this warp's kRing barriers
   uint32_t count;       // segments this warp has streamed (all passes)
   bool dead;            // a ring wait expired: the stream delivers fill values
+  uint32_t* status;     // TV_DEV_TIMEOUT is raised there when a wait expires
 };
 
 __device__ __forceinline__ void seg_issue(const SegStream& st, int sl, uint32_t stage) {
@@ -283,8 +284,11 @@ __device__ __forceinline__ void stream_pass(SegStream& st, float zfill, F&& f) {
     return;
   }
   const uint32_t c0 = st.count;
-  if (lane == 0 && !st.dead)
+  if (lane == 0 && !st.dead) {
+    // the previous pass's generic reads of the ring come before these copies
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     for (int i = 0; i < min(kRing, ns); ++i) seg_issue(st, warp + i * kAcceptWarps, (c0 + i) % kRing);
+  }
   for (int i = 0; i < ns; ++i) {
     const uint32_t g = c0 + i, stage = g % kRing;
     const int sl = warp + i * kAcceptWarps;
@@ -292,6 +296,7 @@ __device__ __forceinline__ void stream_pass(SegStream& st, float zfill, F&& f) {
     if (!st.dead && !__all_sync(0xffffffffu, ring_wait(st.bar + stage, (g / kRing) & 1))) {
       // expired: issue nothing more, let the copies in flight land (bounded)
       st.dead = true;
+      if (lane == 0) set_status(st.status, TV_DEV_TIMEOUT);
       if (lane == 0)
         for (int j = i; j < min(i + kRing, ns); ++j) ring_wait(st.bar + (c0 + j) % kRing, ((c0 + j) / kRing) & 1);
       __syncwarp();
@@ -616,6 +621,7 @@ accept_node_kernel(AcceptParams p) {
   st.bar = sh.ring_bar + warp * kRing;
   st.count = 0;
   st.dead = false;
+  st.status = p.status;
   if (st.bulk) {
     if (lane == 0) {
       for (int r = 0; r < kRing; ++r)
