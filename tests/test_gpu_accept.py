@@ -164,3 +164,47 @@ def test_specexec70b_accept(temperature, mode):
     g, o, st = _run(case)
     exact, near = check_accept(g, o, case.parent, c["T"])
     assert exact + near == 1
+
+
+@pytest.mark.parametrize("V,noise", [(6, 0.7), (600, 1.5)])
+def test_first_token_distribution_over_many_sequences(V, noise):
+    """Speculative sampling is lossless: over sequences whose children are
+    drawn i.i.d. from q, the first emitted token (the accepted child's token,
+    else the residual sample) follows softmax(z_root / tau) exactly (SpecExec
+    page, "Builds on": speculative sampling reproduces the target's
+    distribution).  One call carries 16384 sequences, each with its own
+    Philox stream; 8 seeds give 131072 samples, compared with the closed form
+    by a chi-square test (bins with an expected count below 40 pooled).  V =
+    600 runs two-CTA clusters and residual passes over two segments."""
+    import scipy.stats
+    import tree_verification_verify_b200 as tv
+    tau, T, B = 0.9, 5, 16384
+    par = np.array([-1, 0, 0, 0, 1], dtype=np.int32)
+    base = accept_case(1, T, V, par, tau, sigma=1.0, seed=21, correlated=True, noise=noise)
+    z = base.target_logits.expand(B, T, V).contiguous().cuda()
+    q = base.draft_probs.expand(B, T, V).contiguous().cuda()
+    parent = torch.from_numpy(np.broadcast_to(par, (B, T)).copy()).cuda()
+    qd = base.draft_probs[0].double()
+    gen = torch.Generator().manual_seed(22)
+    p = torch.softmax(base.target_logits[0, 0].double() / float(np.float32(tau)), -1).numpy()
+    counts = np.zeros(V)
+    rounds = 8
+    for s in range(rounds):
+        tok = torch.zeros(B, T, dtype=torch.int32)
+        for j in range(1, T):
+            tok[:, j] = torch.multinomial(qd[par[j]], B, replacement=True, generator=gen).to(torch.int32)
+        g = tv.tree_accept(z, tok.cuda(), parent, draft_probs=q, mode="specsample", temperature=tau,
+                           seed=1000 + s, step=0)
+        first = g["out_tokens"][:, 0].cpu().numpy()
+        assert first.min() >= 0 and first.max() < V
+        counts += np.bincount(first, minlength=V)
+    n = rounds * B
+    expect = n * p
+    big = expect >= 40.0
+    obs = np.append(counts[big], counts[~big].sum())
+    exp = np.append(expect[big], expect[~big].sum())
+    if exp[-1] == 0.0:
+        obs, exp = obs[:-1], exp[:-1]
+    chi2 = float(np.sum((obs - exp) ** 2 / exp))
+    dof = len(obs) - 1
+    assert chi2 < scipy.stats.chi2.isf(1e-4, dof), (chi2, dof)
