@@ -248,8 +248,8 @@ struct SegStream {
   uint32_t ring;        // shared address of this warp's ring
   uint64_t* bar;        // this warp's kRing barriers
   uint32_t count;       // segments this warp has streamed (all passes)
-  bool dead;            // a ring wait expired: the stream delivers fill values
-  uint32_t* status;     // TV_DEV_TIMEOUT is raised there when a wait expires
+  bool dead;            // a ring wait expired: the stream delivers fill values,
+                        // and the kernel raises TV_DEV_TIMEOUT before it exits
 };
 
 __device__ __forceinline__ void seg_issue(const SegStream& st, int sl, uint32_t stage) {
@@ -284,11 +284,8 @@ __device__ __forceinline__ void stream_pass(SegStream& st, float zfill, F&& f) {
     return;
   }
   const uint32_t c0 = st.count;
-  if (lane == 0 && !st.dead) {
-    // the previous pass's generic reads of the ring come before these copies
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (lane == 0 && !st.dead)
     for (int i = 0; i < min(kRing, ns); ++i) seg_issue(st, warp + i * kAcceptWarps, (c0 + i) % kRing);
-  }
   for (int i = 0; i < ns; ++i) {
     const uint32_t g = c0 + i, stage = g % kRing;
     const int sl = warp + i * kAcceptWarps;
@@ -296,7 +293,6 @@ __device__ __forceinline__ void stream_pass(SegStream& st, float zfill, F&& f) {
     if (!st.dead && !__all_sync(0xffffffffu, ring_wait(st.bar + stage, (g / kRing) & 1))) {
       // expired: issue nothing more, let the copies in flight land (bounded)
       st.dead = true;
-      if (lane == 0) set_status(st.status, TV_DEV_TIMEOUT);
       if (lane == 0)
         for (int j = i; j < min(i + kRing, ns); ++j) ring_wait(st.bar + (c0 + j) % kRing, ((c0 + j) / kRing) & 1);
       __syncwarp();
@@ -621,7 +617,6 @@ accept_node_kernel(AcceptParams p) {
   st.bar = sh.ring_bar + warp * kRing;
   st.count = 0;
   st.dead = false;
-  st.status = p.status;
   if (st.bulk) {
     if (lane == 0) {
       for (int r = 0; r < kRing; ++r)
@@ -885,6 +880,8 @@ accept_node_kernel(AcceptParams p) {
       if (tid == 0) p.ticket[b] = 0;           // ready for the next call
     }
   }
+  // a ring wait that expired left this warp's passes on fill values
+  if (st.dead && lane == 0) set_status(p.status, TV_DEV_TIMEOUT);
   cl.sync();                                   // no CTA leaves while others may read its slots
 }
 
