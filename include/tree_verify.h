@@ -222,8 +222,8 @@ TV_API size_t tree_accept_workspace_size(const tv_accept_args* a);
 TV_API tv_status tree_accept(const tv_accept_args* a, void* ws, size_t ws_bytes,
                       tv_stream_t stream);
 
-/* tree_accept without a caller workspace (no counterpart in the paper; an
- * interface addition of this library).  For callers that cannot allocate
+/* tree_accept without a caller workspace (an interface addition of this
+ * library, not a step of the method).  For callers that cannot allocate
  * device memory: code whose device memory is owned by another runtime that
  * reserved it up front (an inference server's pool), or code on a path
  * where cudaMalloc's implicit device-wide synchronisation is not allowed.
