@@ -15,6 +15,10 @@ path computes, written from the method's definitions:
                   (SpecExec page, "Experimental setup": builds on speculative
                   sampling / SpecInfer), and SpecExec's sample-and-descend rule
                   for deterministic trees (SpecExec page, "Approach").
+* commit.py    -- appending the accepted path's K/V to the cache, the step
+                  that makes the accepted tokens prefix for the next
+                  iteration (SpecExec page, "Approach" / "Key results":
+                  accepted tokens per target iteration).
 * expand.py    -- SpecExec's batched best-first (Dijkstra-style) expansion
                   that keeps the highest cumulative-probability continuations
                   (SpecExec page, "Approach"; "Builds on": Dijkstra's
