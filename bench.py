@@ -406,6 +406,55 @@ def time_e2e(step, K, W, flush):
     return tot / K, h2d, d2h
 
 
+def time_commit(step, K, W, flush):
+    """tree_commit_kv on the step's accepted paths (the acceptance outputs of
+    the last step), timed alone from a CUDA graph of its own: the K and V rows
+    of each root and its accepted nodes are appended to a scratch cache of T
+    rows per sequence (prefix_len set to 0 before every call, outside the
+    timed region: where the rows land does not change the work).  Returns
+    (ms per call, bytes moved per call: rows read plus rows written)."""
+    a = step.attn
+    B, T, Hkv, d = a.k_tree.shape
+    kc = torch.zeros(B, T, Hkv, d, dtype=a.k_tree.dtype, device=step.dev)
+    vc = torch.zeros_like(kc)
+    pl = torch.zeros(B, dtype=torch.int32, device=step.dev)
+    n_acc, acc = step.acc_out["n_accepted"], step.acc_out["accepted_nodes"]
+
+    def one():
+        step.tv.tree_commit_kv(kc, vc, pl, a.k_tree, a.v_tree, n_acc, acc, dev_status=step.status)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        pl.zero_()
+        one()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        one()
+    cur = torch.cuda.current_stream()
+    for _ in range(W):
+        flush.zero_()
+        pl.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(K):
+        flush.zero_()
+        pl.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        g.replay()
+        e1.record(cur)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    rows = int((n_acc.clamp(min=0) + 1).sum().item())
+    moved = 2.0 * 2.0 * rows * Hkv * d * a.k_tree.element_size()
+    del g
+    return tot / K, moved
+
+
 # --------------------------------------------------------------------------
 # CPU baseline (the oracle, bounded sample)
 # --------------------------------------------------------------------------
@@ -539,6 +588,8 @@ def main():
     ms_exp = max_over_ranks(statistics.fmean(times["expand"]), world) if "expand" in times else 0.0
     e2e_ms, h2d, d2h = time_e2e(step, max(3, args.steps // 5), 3, flush)
     e2e_ms = max_over_ranks(e2e_ms, world)
+    commit_ms, commit_bytes = time_commit(step, max(3, args.steps), 3, flush)
+    commit_ms = max_over_ranks(commit_ms, world)
     tokens = step.B * step.T * world
     hbm, bf16, bf16_sus, src = peaks()
     # dominant call and its roofline
@@ -594,6 +645,10 @@ def main():
         "gpu_launches": step.launches_per_step() * args.steps,
         "clocks": clocks,
     }
+    # the KV commit of the accepted paths (not part of the timed step)
+    line["calls"]["tree_commit_kv_us"] = round(commit_ms * 1e3, 2)
+    line["calls"]["commit_bytes"] = commit_bytes
+    line["calls"]["commit_gbs"] = round(commit_bytes / (commit_ms * 1e-3) / 1e9, 1)
     if step.expand:
         line["calls"]["tree_expand_us"] = round(ms_exp * 1e3, 2)
         line["calls"]["expand_gbs"] = round(step.expand_bytes / (ms_exp * 1e-3) / 1e9, 1)

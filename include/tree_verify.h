@@ -25,7 +25,11 @@
  *                        (Dijkstra-style) tree construction that keeps the
  *                        highest cumulative-probability continuations
  *                        (SpecExec page, "Approach"; "Builds on": Dijkstra's
- *                        algorithm).
+ *                        algorithm);
+ *   tree_commit_kv    -- the accepted path's K/V appended to the cache, so
+ *                        that the accepted tokens are prefix for the next
+ *                        iteration (SpecExec page, "Approach"; "Key
+ *                        results": accepted tokens per target iteration).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -82,7 +86,8 @@ enum {
   TV_DEV_BAD_PARENT = 1,    /* parent[0] != -1 or parent[i] not in [0, i)  */
   TV_DEV_BAD_TOKEN = 2,     /* a draft token outside [0, V)                */
   TV_DEV_NONFINITE = 4,     /* NaN/Inf logits, or invalid probabilities    */
-  TV_DEV_BAD_ROW = 8,       /* expansion row for a missing/expanded node   */
+  TV_DEV_BAD_ROW = 8,       /* expansion row for a missing/expanded node,  */
+                            /* or a malformed accepted path (commit)       */
   TV_DEV_BAD_LEN = 16,      /* n_nodes or prefix_len out of range          */
   TV_DEV_TIMEOUT = 32       /* a bounded in-kernel wait expired; the       */
                             /* affected outputs are NaN                    */
@@ -288,6 +293,49 @@ TV_API tv_status tree_expand_init(const tv_expand_args* a, int32_t root_token,
                            tv_stream_t stream);
 TV_API tv_status tree_expand_topb(const tv_expand_args* a, void* ws, size_t ws_bytes,
                            tv_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * tree_commit_kv
+ *
+ * Makes the accepted tokens prefix for the next iteration (SpecExec page,
+ * "Approach"; "Key results" count accepted tokens per target iteration;
+ * the pages do not spell out the cache update and this is its plain
+ * reading).  For sequence b with L = prefix_len[b], n = n_accepted[b] and
+ * the path rows = (0, accepted_nodes[b][0], ..., accepted_nodes[b][n-1]) --
+ * the root, then the nodes tree_accept accepted, in path order --
+ *     k_cache[b][L + r][g][:] = k_tree[b][rows[r]][g][:]   (V likewise)
+ * for r = 0 .. n and every kv head g, then prefix_len[b] = L + n + 1.  The
+ * walk's bonus token has no K/V yet: it is the next tree's root.
+ * Every row is read before any row is written, so the tree K/V may be rows
+ * of the cache itself at or after row L of the same sequence (k_tree =
+ * k_cache + L * kv_sl with kt_st = kv_sl, and so on): the accepted rows
+ * are then compacted to the front.  No other overlap between the tree and
+ * the cache, and none between sequences, is allowed.
+ * Layouts (element strides, d contiguous): k_cache, v_cache
+ * [B][Lmax][Hkv][d] (kv_sb, kv_sl, kv_sh) and k_tree, v_tree [B][T][Hkv][d]
+ * (kt_sb, kt_st, kt_sh) as in tree_verify_attn; n_accepted [B] and
+ * accepted_nodes [B][T] (row stride acc_sb) as tree_accept writes them;
+ * prefix_len [B] int32, read and then advanced.  dtype TV_FP32 or TV_BF16,
+ * 1 <= d <= 1024, base pointers aligned to the element size.  No workspace.
+ * Faults: n outside [0, T-1], L outside [0, Lmax] or L + n + 1 > Lmax ->
+ * TV_DEV_BAD_LEN; a path node outside [1, T), or a path that does not
+ * increase -> TV_DEV_BAD_ROW; such a sequence is left as it was (cache and
+ * prefix_len).
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int32_t dtype;
+  int32_t B, T, Hkv, d, Lmax;
+  void* k_cache;
+  void* v_cache;        int64_t kv_sb, kv_sl, kv_sh;
+  int32_t* prefix_len;
+  const void* k_tree;
+  const void* v_tree;   int64_t kt_sb, kt_st, kt_sh;
+  const int32_t* n_accepted;
+  const int32_t* accepted_nodes; int64_t acc_sb;
+  uint32_t* dev_status;
+} tv_commit_args;
+
+TV_API tv_status tree_commit_kv(const tv_commit_args* a, tv_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Utilities

@@ -42,7 +42,7 @@ def test_every_declared_symbol_is_exported(L):
 def test_struct_layouts_match_the_header(L, tmp_path):
     import tree_verification_verify_b200 as tv
     structs = {"tv_attn_args": tv.AttnArgs, "tv_accept_args": tv.AcceptArgs,
-               "tv_expand_args": tv.ExpandArgs}
+               "tv_expand_args": tv.ExpandArgs, "tv_commit_args": tv.CommitArgs}
     src = ['#include <stdio.h>', '#include <stddef.h>', '#include "tree_verify.h"', "int main(void){"]
     for cname, py in structs.items():
         src.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
@@ -90,6 +90,21 @@ def test_host_argument_checks(L):
     assert L.tree_verify_attn(ctypes.byref(at), None, 0, None) == 1
     at.Hq, at.d = 8, 96                                              # d unsupported
     assert L.tree_verify_attn(ctypes.byref(at), None, 0, None) == 2
+    c = tv.CommitArgs()
+    c.dtype, c.B, c.T, c.Hkv, c.d, c.Lmax = 1, 0, 4, 2, 64, 16      # B = 0: nothing to do
+    assert L.tree_commit_kv(ctypes.byref(c), None) == 0
+    c.B = 1                                                          # B > 0 without arrays
+    assert L.tree_commit_kv(ctypes.byref(c), None) == 1
+    c.k_cache = c.v_cache = c.k_tree = c.v_tree = 1024
+    c.prefix_len = c.n_accepted = c.accepted_nodes = 2048
+    c.k_tree = 1025                                                  # not element-aligned
+    assert L.tree_commit_kv(ctypes.byref(c), None) == 1
+    c.k_tree, c.d = 1024, 2048                                       # d > 1024
+    assert L.tree_commit_kv(ctypes.byref(c), None) == 2
+    c.d, c.dtype = 64, 7                                             # unknown dtype
+    assert L.tree_commit_kv(ctypes.byref(c), None) == 1
+    c.dtype, c.T = 1, 0                                              # B > 0 with T = 0
+    assert L.tree_commit_kv(ctypes.byref(c), None) == 1
 
 
 def test_pool_bytes_grow_with_budget(L):

@@ -21,7 +21,7 @@ from typing import Optional
 import torch
 
 __all__ = ["lib", "version", "status_string", "tree_verify_attn", "tree_accept", "tree_accept_noalloc",
-           "tree_expand_init", "tree_expand_topb", "ExpandState", "philox_uniforms",
+           "tree_expand_init", "tree_expand_topb", "ExpandState", "tree_commit_kv", "philox_uniforms",
            "TVError", "MODES"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -71,6 +71,15 @@ class ExpandArgs(ctypes.Structure):
                 ("frontier", c_vp), ("n_appended", c_vp), ("dev_status", c_vp)]
 
 
+class CommitArgs(ctypes.Structure):
+    _fields_ = [("dtype", c_i32), ("B", c_i32), ("T", c_i32), ("Hkv", c_i32), ("d", c_i32), ("Lmax", c_i32),
+                ("k_cache", c_vp), ("v_cache", c_vp), ("kv_sb", c_i64), ("kv_sl", c_i64), ("kv_sh", c_i64),
+                ("prefix_len", c_vp),
+                ("k_tree", c_vp), ("v_tree", c_vp), ("kt_sb", c_i64), ("kt_st", c_i64), ("kt_sh", c_i64),
+                ("n_accepted", c_vp), ("accepted_nodes", c_vp), ("acc_sb", c_i64),
+                ("dev_status", c_vp)]
+
+
 class TVError(RuntimeError):
     pass
 
@@ -91,6 +100,7 @@ def lib() -> ctypes.CDLL:
                            ("tree_accept_noalloc", [ctypes.POINTER(AcceptArgs), c_vp]),
                            ("tree_expand_topb", [ctypes.POINTER(ExpandArgs), c_vp, c_size, c_vp]),
                            ("tree_expand_init", [ctypes.POINTER(ExpandArgs), c_i32, c_vp]),
+                           ("tree_commit_kv", [ctypes.POINTER(CommitArgs), c_vp]),
                            ("tv_philox_uniforms", [c_u64, c_u64, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp])):
             f = getattr(L, name)
             f.argtypes = args
@@ -241,6 +251,46 @@ last_attn_path = None
 last_attn_launches = None
 ATTN_PATHS = {0: "cuda-core split-KV", 1: "tcgen05 prefix", 2: "block top-k sparse (cuda cores)",
               3: "block top-k sparse (tcgen05)"}
+
+
+# --------------------------------------------------------------- KV commit
+
+def tree_commit_kv(k_cache, v_cache, prefix_len, k_tree, v_tree, n_accepted, accepted_nodes,
+                   dev_status=None, stream=None):
+    """Append each sequence's accepted path (the root, then the accepted
+    nodes) to its K/V cache and advance prefix_len in place
+    (include/tree_verify.h, tree_commit_kv).  Shapes: caches [B][Lmax][Hkv][d],
+    tree K/V [B][T][Hkv][d] (may be a view of the cache rows from
+    prefix_len on), prefix_len and n_accepted [B] int32, accepted_nodes
+    [B][T] int32 as tree_accept returns them."""
+    dev = _need_cuda(k_cache, v_cache, prefix_len, k_tree, v_tree, n_accepted, accepted_nodes, dev_status)
+    if k_cache.dtype == torch.bfloat16:
+        dt = TV_BF16
+    elif k_cache.dtype == torch.float32:
+        dt = TV_FP32
+    else:
+        raise TVError("K/V must be bf16 or fp32")
+    for t in (k_cache, v_cache, k_tree, v_tree):
+        if t.dtype != k_cache.dtype or t.stride(-1) != 1:
+            raise TVError("K/V must share one dtype with a contiguous last dimension")
+    if k_cache.stride() != v_cache.stride() or k_tree.stride() != v_tree.stride():
+        raise TVError("K and V tensors must have equal strides")
+    B, Lmax, Hkv, d = k_cache.shape
+    T = k_tree.shape[1]
+    if tuple(k_tree.shape) != (B, T, Hkv, d) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise TVError("tree K/V must be [B][T][Hkv][d] and match the caches")
+    prefix_len = _i32(prefix_len)
+    n_accepted = _i32(n_accepted)
+    if accepted_nodes.dtype != torch.int32 or accepted_nodes.stride(-1) != 1:
+        raise TVError("accepted_nodes must be int32 with contiguous rows")
+    a = CommitArgs(dt, B, T, Hkv, d, Lmax,
+                   k_cache.data_ptr(), v_cache.data_ptr(), k_cache.stride(0), k_cache.stride(1), k_cache.stride(2),
+                   prefix_len.data_ptr(),
+                   k_tree.data_ptr(), v_tree.data_ptr(), k_tree.stride(0), k_tree.stride(1), k_tree.stride(2),
+                   n_accepted.data_ptr(), accepted_nodes.data_ptr(), accepted_nodes.stride(0),
+                   _ptr(dev_status))
+    _check(lib().tree_commit_kv(ctypes.byref(a), _stream(stream)), "tree_commit_kv")
+    return prefix_len
 
 
 # --------------------------------------------------------------- acceptance

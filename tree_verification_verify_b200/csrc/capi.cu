@@ -21,6 +21,7 @@ cudaError_t launch_block_means(const AttnParams& p, float* kbar, cudaStream_t st
 cudaError_t launch_block_select(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attn_sparse(const AttnParams& p, cudaStream_t stream);
 int num_sms();
+cudaError_t launch_commit(const tv_commit_args* a, cudaStream_t stream);
 }  // namespace tv
 
 using namespace tv;
@@ -304,6 +305,36 @@ extern "C" tv_status tree_expand_topb(const tv_expand_args* a, void*, size_t, tv
   const tv_status st = check_expand(a, true);
   if (st != TV_OK) return st;
   return from_cuda(launch_expand(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// ------------------------------------------------------------ KV commit
+
+namespace {
+tv_status check_commit(const tv_commit_args* a) {
+  if (!a) return TV_ERR_INVALID_ARG;
+  if (a->dtype != TV_FP32 && a->dtype != TV_BF16) return TV_ERR_INVALID_ARG;
+  if (a->B < 0 || a->T < 0 || a->Hkv <= 0 || a->Lmax < 0 || a->d < 1) return TV_ERR_INVALID_ARG;
+  if (a->d > 1024) return TV_ERR_UNSUPPORTED;
+  if (a->B > 0) {
+    if (a->T < 1) return TV_ERR_INVALID_ARG;
+    if (!a->k_cache || !a->v_cache || !a->prefix_len || !a->k_tree || !a->v_tree || !a->n_accepted)
+      return TV_ERR_INVALID_ARG;
+    if (a->T > 1 && !a->accepted_nodes) return TV_ERR_INVALID_ARG;
+    const uintptr_t es = a->dtype == TV_BF16 ? 2u : 4u;
+    const uintptr_t ptrs[4] = {reinterpret_cast<uintptr_t>(a->k_cache), reinterpret_cast<uintptr_t>(a->v_cache),
+                               reinterpret_cast<uintptr_t>(a->k_tree), reinterpret_cast<uintptr_t>(a->v_tree)};
+    for (uintptr_t x : ptrs)
+      if (x % es != 0) return TV_ERR_INVALID_ARG;
+  }
+  return TV_OK;
+}
+}  // namespace
+
+extern "C" tv_status tree_commit_kv(const tv_commit_args* a, tv_stream_t stream) {
+  const tv_status st = check_commit(a);
+  if (st != TV_OK) return st;
+  if (a->B == 0) return TV_OK;
+  return from_cuda(launch_commit(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 // ------------------------------------------------------------ utilities
