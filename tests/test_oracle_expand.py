@@ -5,6 +5,11 @@
   enumerated to a depth that contains it.
 * Bsel > 1 equals an independent heap-based simulation of the rounds that
   keeps every candidate (so pool truncation loses nothing).
+* Ties: with every logit of a row equal, all candidates of one depth tie
+  exactly and the order rests on the tie-breaks alone (parent ascending,
+  then token ascending): the oracle equals the heap simulation (which
+  orders by the tuple (-score, parent, token)), and at Bsel = 1 the tree is
+  the breadth-first numbering (node k: parent (k-1) // V, token (k-1) % V).
 * Best-first differs from beam search (the SpecExec page's ablation) and,
   at Bsel = 1, keeps at least as much draft probability mass.
 * A closed-form worked example with exact probabilities (golden file).
@@ -73,15 +78,16 @@ def test_bsel1_is_global_top_n(seed):
         assert abs(st.logp[i] - allp[p]) < 1e-12
 
 
-def _heap_rounds(V, Bsel, budget, sigma, seed):
+def _heap_rounds(V, Bsel, budget, sigma, seed, rows=None):
     """Independent round simulation: a binary heap over every candidate
-    ever generated (no truncation)."""
+    ever generated (no truncation).  rows(path) gives a node's draft
+    logits (default: the seeded Gaussian rows)."""
     paths, logp, par, tok = [()], [0.0], [-1], [0]
     heap = []
     frontier = [0]
     while len(paths) < budget and frontier:
         for n in frontier:
-            z = _row(paths[n], V, sigma, seed)
+            z = rows(paths[n]) if rows else _row(paths[n], V, sigma, seed)
             lz = z - logsumexp(z)
             for t in range(V):
                 heapq.heappush(heap, (-(logp[n] + lz[t]), n, t))
@@ -105,6 +111,22 @@ def test_batched_rounds_match_heap_simulation(V, Bsel, budget, seed):
     assert st.parent == par and st.token == tok
     np.testing.assert_allclose(st.logp, logp, rtol=0, atol=1e-12)
     assert min(st.gaps) > 1e-9     # no near-ties decided these seeds
+
+
+@pytest.mark.parametrize("V,Bsel,budget", [(2, 3, 40), (3, 1, 30), (4, 5, 50), (5, 2, 33), (7, 16, 64)])
+def test_ties_order_by_parent_then_token(V, Bsel, budget):
+    def flat(path):
+        return np.full(V, 0.25 * len(path))
+    st = ExpandState(budget)
+    frontier = [0]
+    while st.n_nodes < budget and frontier:
+        paths = _paths(st)
+        frontier = expand_call(st, np.stack([flat(paths[n]) for n in frontier]), frontier, Bsel)
+    par, tok, _ = _heap_rounds(V, Bsel, budget, 0.0, 0, rows=flat)
+    assert st.parent == par and st.token == tok
+    if Bsel == 1:
+        k = np.arange(1, budget)
+        assert st.parent[1:] == list((k - 1) // V) and st.token[1:] == list((k - 1) % V)
 
 
 def _beam(V, Bsel, budget, rows):
