@@ -1,26 +1,36 @@
 """Benchmark of the tree-verification hot path on B200.
 
-One step = one pass of the verification path over one batch of the
-Llama-3-8B-shaped workload (batch 1, 32 query / 8 kv heads, d = 128, bf16,
-4096-token prefix, 64-node tree, vocabulary 128256, temperature 0.8):
-tree-masked attention of the 64 nodes (tree_verify_attn) followed by the
-speculative-sampling acceptance walk (tree_accept).  `value` is verified
-tree tokens per second per layer over all ranks.  Inputs are synthetic
-(seeded Gaussian activations and logits of those shapes).
+Default workload: the long-context configuration, the largest one that fits a
+single GPU -- batch 4, 32 query / 8 kv heads, d = 128, bf16, a 131072-token
+prefix per sequence, a 256-node draft tree, vocabulary 128256, temperature 0.
+One step = tree-masked attention of the 4 x 256 nodes over prefix and
+ancestors (tree_verify_attn, dense) followed by the greedy acceptance walk
+(tree_accept).  `value` is verified tree tokens per second per layer over all
+ranks.  Inputs are synthetic (seeded Gaussian activations and logits of those
+shapes).
+
+The same run then times the other named workloads, each as its own step, and
+reports them under "configs" in the same JSON line: block top-k long context
+(the sparse path), the SpecExec-shaped 2048-node tree (16 rounds of
+tree_expand_topb build it on the device, then attention and SpecExec
+acceptance), batched serving (32 sequences) and the Llama-3-8B layer.  Every
+call carries its roofline fraction against the measured peaks and against
+the 8 TB/s / 2.25 PFLOP/s denominators.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--config llama3_8b|specexec70b|serving|longctx|longctx_sparse|tiny]
+                    [--config longctx|longctx_sparse|specexec70b|serving|llama3_8b|tiny]
+                    [--only] [--no-cpu-baseline]
 
 Timing: the step's calls are captured once into one CUDA graph (and each
 call into a graph of its own); W untimed warm-up steps, then K steps of the
 one-graph step, each preceded (outside the timed region) by a 256 MiB write
 that flushes the 126 MB L2 and bracketed by CUDA events on the launching
 stream (`ms_per_step`, `value`); then K steps of the per-call graphs with an
-event between calls give the per-call durations (`calls`); the max over
-ranks is reported.  The e2e figure calls
-the Python API directly (no graph), copying the step's inputs from pinned
-host memory and reading the accepted tokens back.  --impl reference times
-the fp64 CPU oracle on a bounded sample of the same workload.
+event between calls give the per-call durations; the max over ranks is
+reported.  The e2e figure calls the Python API directly (no graph), copying
+the step's inputs from pinned host memory and reading the accepted tokens
+back.  --impl reference times the fp64 CPU oracle on a bounded sample of the
+same workload, spread over the host cores by a process pool.
 """
 
 from __future__ import annotations
@@ -43,12 +53,20 @@ sys.path.insert(0, ROOT)
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+# the denominators the targets are stated against: 8 TB/s HBM and the B200
+# dense bf16 datasheet peak
+TARGET_HBM_GBS = 8000.0
+TARGET_BF16_TFLOPS = 2250.0
 
+CONFIG_NAMES = ["longctx", "longctx_sparse", "specexec70b", "serving", "llama3_8b", "tiny"]
+# the workloads a default run times after its main one
+EXTRA_CONFIGS = ["longctx_sparse", "specexec70b", "serving", "llama3_8b"]
 
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic.txt")
 KERNEL_SOURCES = {
     "accept_node_kernel": "tree_verification_verify_b200/csrc/accept.cu",
     "attn_tc_kernel": "tree_verification_verify_b200/csrc/attn_tc.cu",
+    "attn_pair_kernel": "tree_verification_verify_b200/csrc/attn_pair.cu",
     "expand_rows_kernel": "tree_verification_verify_b200/csrc/expand.cu",
 }
 
@@ -81,6 +99,18 @@ def peaks():
         return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def roofline_fracs(seconds, nbytes=0.0, flops=0.0):
+    """Roofline fraction of one call: (the slower of bytes / HBM bandwidth and
+    FLOPs / bf16 peak) / measured time, against the measured peaks and
+    against the 8 TB/s / 2.25 PFLOP/s denominators."""
+    hbm, bf16, _, _ = peaks()
+    out = {}
+    for key, bw, pk in (("frac_measured", hbm, bf16), ("frac_target", TARGET_HBM_GBS, TARGET_BF16_TFLOPS)):
+        t = max(nbytes / (bw * 1e9), flops / (pk * 1e12))
+        out[key] = round(t / seconds, 4) if seconds > 0 else None
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -185,7 +215,41 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------
-# workloads
+# algorithmic work
+# --------------------------------------------------------------------------
+
+def attn_work(parents, prefix_lens, T, Hq, Hkv, d, elt, kept_keys=None, union_blocks=None,
+              block_size=64, means_in_call=False):
+    """Algorithmic FLOPs and bytes of one tree_verify_attn call.
+
+    FLOPs = 4 d Hq sum_i |K(i)| (QK^T and PV), |K(i)| = prefix keys (dense) or
+    kept keys (block top-k, per kv head) plus the root path.  Bytes = every
+    K/V element read once: the prefix (dense) or, for block top-k, the union
+    over a sequence's nodes of the kept blocks per kv head, plus one K read
+    for the block means when they are computed in the call; and the tree
+    K/V rows."""
+    from synth import tree_depths
+    B = len(prefix_lens)
+    G = Hq // Hkv
+    path = 0
+    for b in range(B):
+        path += int(np.sum(tree_depths(np.asarray(parents[b])) + 1))
+    tree_bytes = float(B * T) * Hkv * d * 2 * elt
+    if kept_keys is None:
+        keys = sum(T * int(L) for L in prefix_lens)
+        flops = 4.0 * d * Hq * (keys + path)
+        nbytes = float(sum(int(L) for L in prefix_lens)) * Hkv * d * 2 * elt + tree_bytes
+    else:
+        # kept_keys: total kept prefix keys over (b, node, kv head)
+        flops = 4.0 * d * G * kept_keys + 4.0 * d * Hq * path
+        nbytes = float(union_blocks) * block_size * d * 2 * elt + tree_bytes
+        if means_in_call:
+            nbytes += float(sum(int(L) for L in prefix_lens)) * Hkv * d * elt
+    return flops, nbytes
+
+
+# --------------------------------------------------------------------------
+# workloads (device side: the library path)
 # --------------------------------------------------------------------------
 
 class Step:
@@ -198,7 +262,7 @@ class Step:
 
     def __init__(self, name, seed, dev):
         import tree_verification_verify_b200 as tv
-        from synth import CONFIGS, config_attn_case, config_accept_case, config_expand_case, tree_depths
+        from synth import CONFIGS, config_attn_case, config_accept_case, config_expand_case
         self.tv = tv
         self.name = name
         base = "longctx" if name == "longctx_sparse" else name
@@ -241,19 +305,18 @@ class Step:
                             min_margin=torch.empty(B, dtype=torch.float64, device=dev))
         # algorithmic work
         Hkv = self.attn.k_cache.shape[2]
-        L = self.attn.prefix_len.cpu().numpy()
+        L = [int(x) for x in self.attn.prefix_len.cpu().numpy()]
         par = self.attn.parent.cpu().numpy()
-        keys = 0
-        for b in range(B):
-            dep = tree_depths(par[b])
-            Lb = int(L[b])
-            if self.sparse:
-                nblk = (Lb + 63) // 64
-                Lb = min(Lb, 32 * 64) if nblk > 32 else Lb
-            keys += T * Lb + int(np.sum(dep + 1))
         elt = self.attn.q.element_size()
-        self.attn_flops = 4.0 * d * Hq * keys
-        self.attn_bytes = float(sum(int(x) + T for x in L)) * Hkv * d * 2 * elt
+        self.union_blocks = None
+        if self.sparse:
+            kept, union = self.measure_selection()
+            self.union_blocks = union
+            self.attn_flops, self.attn_bytes = attn_work(par, L, T, Hq, Hkv, d, elt, kept_keys=kept,
+                                                         union_blocks=union, block_size=self.attn.block_size,
+                                                         means_in_call=True)
+        else:
+            self.attn_flops, self.attn_bytes = attn_work(par, L, T, Hq, Hkv, d, elt)
         V = self.acc.target_logits.shape[2]
         internal = 0
         if self.acc.draft_probs is not None:
@@ -263,6 +326,28 @@ class Step:
         self.expand_bytes = 0.0
         if self.expand:
             self.expand_bytes = float(sum(x.numel() for x in self.exp_logits) * 4)
+
+    def measure_selection(self):
+        """Kept prefix keys summed over (sequence, node, kv head) and the
+        number of distinct kept blocks summed over (sequence, kv head), from
+        the selection the library returns (one untimed call)."""
+        a = self.attn
+        _, _, sel = self.tv.tree_verify_attn(a.q, a.k_cache, a.v_cache, a.prefix_len, a.k_tree, a.v_tree,
+                                             a.parent, sparse_topk=a.sparse_topk, block_size=a.block_size,
+                                             want_sel=True)
+        torch.cuda.synchronize()
+        sel = sel.cpu().numpy()                     # [B][T][Hkv][k]
+        L = a.prefix_len.cpu().numpy()
+        bs = a.block_size
+        kept, union = 0, 0
+        for b in range(sel.shape[0]):
+            for g in range(sel.shape[2]):
+                s = sel[b, :, g, :]
+                s = s[s >= 0]
+                keys = np.minimum(bs, int(L[b]) - bs * s)
+                kept += int(np.sum(keys))
+                union += len(np.unique(s))
+        return kept, union
 
     def run_expand(self):
         tv, st, ec = self.tv, self.exp_state, self.ec
@@ -287,6 +372,18 @@ class Step:
         attn = self.attn_launches
         exp = (1 + 2 * len(self.exp_logits)) if self.expand else 0
         return attn + 1 + exp
+
+    def near_threshold(self):
+        """Sequences whose walk met a decision within 1e-6 of its threshold
+        (min_margin of the last acceptance call)."""
+        mm = self.acc_out["min_margin"].cpu().numpy()
+        return int(np.sum(mm < 1e-6))
+
+    def free(self):
+        for k in list(self.__dict__):
+            if k not in ("name", "c", "B", "T", "sparse", "expand", "temperature"):
+                self.__dict__.pop(k)
+        torch.cuda.empty_cache()
 
 
 def capture_graphs(step):
@@ -403,6 +500,7 @@ def time_e2e(step, K, W, flush):
         e1.record(s)
         e1.synchronize()
         tot += e0.elapsed_time(e1)
+    del host_in
     return tot / K, h2d, d2h
 
 
@@ -455,64 +553,313 @@ def time_commit(step, K, W, flush):
     return tot / K, moved
 
 
+def call_summary(step, times, world):
+    """Per-call mean times (max over ranks) with their work and roofline
+    fractions."""
+    ms = {nm: max_over_ranks(statistics.fmean(times[nm]), world) for nm in times}
+    out = {"ms_per_step": round(ms["step"], 5),
+           "tree_tokens_per_s": step.B * step.T * world / (ms["step"] * 1e-3)}
+    t = ms["attn"] * 1e-3
+    out["tree_verify_attn"] = {
+        "us": round(ms["attn"] * 1e3, 2), "path": step.attn_path, "launches": step.attn_launches,
+        "tflops": round(step.attn_flops / t / 1e12, 2), "gbs": round(step.attn_bytes / t / 1e9, 1),
+        "algorithmic_flops": step.attn_flops, "algorithmic_bytes": step.attn_bytes,
+        "tokens_per_s": step.B * step.T / t, **roofline_fracs(t, step.attn_bytes, step.attn_flops)}
+    if step.union_blocks is not None:
+        out["tree_verify_attn"]["kept_block_union"] = step.union_blocks
+    t = ms["accept"] * 1e-3
+    out["tree_accept"] = {
+        "us": round(ms["accept"] * 1e3, 2), "mode": step.acc.mode if step.temperature > 0 else "greedy",
+        "gbs": round(step.accept_bytes / t / 1e9, 1), "algorithmic_bytes": step.accept_bytes,
+        "nodes_per_s": step.B * step.T / t, "near_threshold": step.near_threshold(),
+        **roofline_fracs(t, step.accept_bytes)}
+    if "expand" in ms:
+        t = ms["expand"] * 1e-3
+        n_new = step.ec.budget - 1
+        out["tree_expand_topb"] = {
+            "us": round(ms["expand"] * 1e3, 2), "rounds": len(step.exp_logits),
+            "gbs": round(step.expand_bytes / t / 1e9, 1), "algorithmic_bytes": step.expand_bytes,
+            "nodes_per_s": n_new / t, **roofline_fracs(t, step.expand_bytes)}
+    return ms, out
+
+
 # --------------------------------------------------------------------------
-# CPU baseline (the oracle, bounded sample)
+# CPU baseline and reference arm: the fp64 oracle over the host cores
 # --------------------------------------------------------------------------
 
-def cpu_baseline(step, budget_s=15.0):
-    """Time the fp64 oracle on a bounded sample of the step: attention of a
-    subset of nodes (all heads) plus the full acceptance walk; scaled to
-    tokens per second of the whole step."""
-    from oracle.attention import tree_verify_attn as o_attn
-    from oracle.accept import tree_accept as o_accept
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count() or 1
-    a = step.attn
-    c = step.acc
-    host = {k: getattr(a, k).cpu() for k in ("q", "k_cache", "v_cache", "prefix_len", "k_tree", "v_tree", "parent")}
-    ch = dict(z=c.target_logits.cpu(), q=None if c.draft_probs is None else c.draft_probs.cpu(),
-              tok=c.draft_tokens.cpu(), par=c.parent.cpu())
+_POOL = None
+
+
+def _pool_init(files, meta):
+    global _POOL
+    import numpy
+    _POOL = {"meta": meta, "arr": {k: numpy.load(v, mmap_mode="r") for k, v in files.items()}}
+    import oracle.attention  # noqa: F401  (imported before any timing)
+    import oracle.accept  # noqa: F401
+
+
+def _pool_ping(_):
+    return os.getpid()
+
+
+def _as_tensor(a, bf16):
+    x = torch.from_numpy(np.array(a))
+    return x.view(torch.bfloat16) if bf16 else x
+
+
+def _pool_attn(task):
+    """Oracle attention of some nodes of one (sequence, kv head): the call
+    gets that sequence's inputs restricted to the kv head and its G query
+    heads (contiguous GQA groups make this the same arithmetic)."""
+    from oracle.attention import tree_verify_attn
+    b, g, nodes = task
+    A, m = _POOL["arr"], _POOL["meta"]
+    G, bf = m["G"], m["bf16"]
+    q = _as_tensor(A["q"][b:b + 1, :, g * G:(g + 1) * G], bf)
+    k = _as_tensor(A["k"][b, g][None, :, None, :], bf)
+    v = _as_tensor(A["v"][b, g][None, :, None, :], bf)
+    kt = _as_tensor(A["kt"][b, :, g][None, :, None, :], bf)
+    vt = _as_tensor(A["vt"][b, :, g][None, :, None, :], bf)
+    pl = np.asarray(A["pl"][b:b + 1])
+    par = np.asarray(A["par"][b:b + 1])
     t0 = time.perf_counter()
-    o_accept(ch["z"], ch["q"], ch["tok"], ch["par"], mode=c.mode, temperature=step.temperature, seed=c.seed)
-    t_acc = time.perf_counter() - t0
-    t_exp, exp_note = 0.0, ""
-    if step.expand:
-        # expansion: the first calls of the build (all 16 take about as long
-        # as each other past the first), scaled to the whole build
+    tree_verify_attn(q, k, v, pl, kt, vt, par, sparse_topk=m["topk"], block_size=m["bs"],
+                     rows={(0, int(i)) for i in nodes})
+    return time.perf_counter() - t0, len(nodes)
+
+
+def _pool_accept(b):
+    """Oracle acceptance walk of sequence b."""
+    from oracle.accept import tree_accept
+    A, m = _POOL["arr"], _POOL["meta"]
+    z = A["z"][b:b + 1]
+    qd = A["qd"][b:b + 1] if "qd" in A else None
+    tok, par = np.asarray(A["tok"][b:b + 1]), np.asarray(A["par"][b:b + 1])
+    t0 = time.perf_counter()
+    tree_accept(z, qd, tok, par, mode=m["mode"], temperature=m["temp"], seed=m["seed"])
+    return time.perf_counter() - t0
+
+
+class OracleRunner:
+    """Times the fp64 oracle on a workload, spread over the host cores.
+
+    The workload's inputs are written once to temporary .npy files (K/V as
+    [B][Hkv][L][d], bf16 kept as raw 16-bit words) that every worker maps.
+    Attention work is split into tasks of (sequence, kv head, nodes); the
+    acceptance walk into one task per sequence.  Workers are spawned (not
+    forked) with one BLAS thread each; the pool size is the number of cores
+    this process may run on, at most MAX_WORKERS (each worker holds a few
+    hundred MB of fp64 copies of one sequence's K/V)."""
+
+    MAX_WORKERS = 32
+
+    def __init__(self, host, workers=None):
+        self.h = host
+        self.dir = tempfile.mkdtemp(prefix="tv_oracle_")
+        bf = host["q"].dtype == torch.bfloat16
+
+        def arr(t):
+            if isinstance(t, torch.Tensor):
+                t = t.contiguous()
+                return t.view(torch.int16).numpy() if t.dtype == torch.bfloat16 else t.numpy()
+            return np.asarray(t)
+
+        files = {}
+        for name, t in (("q", host["q"]), ("k", host["k_cache"].permute(0, 2, 1, 3)),
+                        ("v", host["v_cache"].permute(0, 2, 1, 3)), ("kt", host["k_tree"]),
+                        ("vt", host["v_tree"]), ("pl", host["prefix_len"]), ("par", host["parent"]),
+                        ("z", host["z"]), ("tok", host["tok"]), ("qd", host["qd"])):
+            if t is None:
+                continue
+            p = os.path.join(self.dir, name + ".npy")
+            np.save(p, arr(t))
+            files[name] = p
+        B, T, Hq, d = host["q"].shape
+        Hkv = host["k_cache"].shape[2]
+        self.B, self.T, self.Hkv, self.G = B, T, Hkv, Hq // Hkv
+        self.meta = dict(G=self.G, bf16=bf, topk=host["topk"], bs=host["bs"], mode=host["mode"],
+                         temp=host["temp"], seed=host["seed"])
+        self.files = files
+        try:
+            ncpu = len(os.sched_getaffinity(0))
+        except Exception:
+            ncpu = os.cpu_count() or 1
+        self.workers = workers or min(ncpu, self.MAX_WORKERS)
+        import multiprocessing as mp
+        saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+        for k in saved:
+            os.environ[k] = "1"
+        try:
+            self.pool = mp.get_context("spawn").Pool(self.workers, initializer=_pool_init,
+                                                     initargs=(files, self.meta))
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        self.pool.map(_pool_ping, range(self.workers))        # every worker is up
+
+    def attn_tasks(self, chunk):
+        """(sequence, kv head, node chunk) tasks, chunk-major so that a prefix
+        of the list covers every (sequence, kv head)."""
+        tasks = []
+        for c0 in range(0, self.T, chunk):
+            for b in range(self.B):
+                for g in range(self.Hkv):
+                    tasks.append((b, g, list(range(c0, min(self.T, c0 + chunk)))))
+        return tasks
+
+    def one_worker_node_seconds(self, nodes=2):
+        """Seconds per (node, kv head) of one oracle call in this process on
+        one thread (the 1-worker time; also sizes the tasks)."""
+        global _POOL
+        from threadpoolctl import threadpool_limits
+        _pool_init(self.files, self.meta)
+        nt = torch.get_num_threads()
+        torch.set_num_threads(1)
+        try:
+            with threadpool_limits(1):
+                dt, n = _pool_attn((0, 0, list(range(min(nodes, self.T)))))
+        finally:
+            torch.set_num_threads(nt)
+            _POOL = None
+        return dt / n
+
+    def time_attention(self, budget_s, per_unit_s):
+        """Wall seconds of the pool over a bounded sample of attention tasks,
+        and the (node, kv head) units it covered."""
+        work_per_worker = max(1, int(budget_s / max(per_unit_s, 1e-6)))
+        chunk = max(1, min(self.T, work_per_worker // 2))
+        tasks = self.attn_tasks(chunk)
+        total_units_wanted = work_per_worker * self.workers
+        sample, units = [], 0
+        for t in tasks:
+            if units >= total_units_wanted:
+                break
+            sample.append(t)
+            units += len(t[2])
+        t0 = time.perf_counter()
+        res = self.pool.map(_pool_attn, sample, chunksize=1)
+        wall = time.perf_counter() - t0
+        return wall, sum(n for _, n in res), sample
+
+    def time_accept(self, seqs):
+        """(wall seconds of the pool, summed seconds of the tasks) for the
+        acceptance walks of the given sequences."""
+        t0 = time.perf_counter()
+        res = self.pool.map(_pool_accept, seqs, chunksize=1)
+        return time.perf_counter() - t0, float(sum(res))
+
+    def close(self):
+        import shutil
+        try:
+            self.pool.terminate()
+            self.pool.join()
+        finally:
+            shutil.rmtree(self.dir, ignore_errors=True)
+
+
+def host_inputs(name, seed=0, device_step=None):
+    """Host copies of a workload's inputs for the oracle.  From the device
+    step when one exists (our arm's CPU baseline), else built on the host
+    from the same seeded generators (the reference arm, which imports
+    nothing of the library: the SpecExec tree is then built by the oracle's
+    own expansion)."""
+    from synth import CONFIGS, config_attn_case, config_accept_case, config_expand_case
+    base = "longctx" if name == "longctx_sparse" else name
+    c = CONFIGS[base]
+    sparse = name == "longctx_sparse"
+    temp = c.get("temperature", c.get("temperatures", (0.0,))[-1])
+    if device_step is not None:
+        a, ac = device_step.attn, device_step.acc
+        h = {k: getattr(a, k).cpu() for k in ("q", "k_cache", "v_cache", "prefix_len", "k_tree", "v_tree",
+                                              "parent")}
+        h.update(z=ac.target_logits.cpu(), tok=ac.draft_tokens.cpu(),
+                 qd=None if ac.draft_probs is None else ac.draft_probs.cpu(), mode=ac.mode, seed=ac.seed,
+                 temp=device_step.temperature, topk=a.sparse_topk, bs=a.block_size,
+                 exp=(device_step.ec, [z.cpu() for z in device_step.exp_logits]) if device_step.expand else None)
+        return h
+    exp = None
+    if base == "specexec70b":
         from oracle.expand import ExpandState as OState, expand_call
-        ec = step.ec
+        ec = config_expand_case(base, seed=seed)
         ost = OState(ec.budget, ec.root_token)
         frontier = [0]
-        n_calls, done_calls, t_e = len(step.exp_logits), 0, 0.0
-        while done_calls < min(3, n_calls):
-            z = step.exp_logits[done_calls].cpu().double().numpy()
-            t0 = time.perf_counter()
-            frontier = list(expand_call(ost, z[:len(frontier)] if done_calls else z[:1],
+        zs = []
+        for call in range(ec.n_calls()):
+            z = ec.round_logits(call, 1 if call == 0 else ec.Bsel)
+            zs.append(z)
+            if not frontier:
+                break
+            frontier = list(expand_call(ost, z.double().numpy()[:len(frontier)],
                                         np.asarray(frontier, np.int64), ec.Bsel))
-            t_e += time.perf_counter() - t0
-            done_calls += 1
-        t_exp = t_e / done_calls * n_calls
-        exp_note = f", plus {done_calls} of {n_calls} expansion rounds scaled to the build"
-    B, T = step.B, step.T
+        par = np.asarray(ost.parent, np.int32)
+        a = config_attn_case(base, seed=seed, parents=[par])
+        ac = config_accept_case(base, temperature=temp, seed=seed, parents=[par], mode="specexec")
+        ac.draft_tokens = torch.tensor(np.asarray(ost.token, np.int32)).view(1, -1)
+        mode = "specexec"
+        exp = (ec, zs)
+    else:
+        a = config_attn_case(base, seed=seed, sparse=sparse)
+        ac = config_accept_case(base, temperature=temp, seed=seed, parents=[p.numpy() for p in a.parent])
+        mode = ac.mode
+    h = {k: getattr(a, k) for k in ("q", "k_cache", "v_cache", "prefix_len", "k_tree", "v_tree", "parent")}
+    h.update(z=ac.target_logits, tok=ac.draft_tokens, qd=ac.draft_probs, mode=mode, seed=ac.seed, temp=temp,
+             topk=a.sparse_topk, bs=a.block_size, exp=exp)
+    return h
+
+
+def time_expand_oracle(exp, rounds=3):
+    """Oracle expansion: the first `rounds` calls of the build timed (each
+    round's rows depend on the previous round), scaled to the whole build."""
+    from oracle.expand import ExpandState as OState, expand_call
+    ec, zs = exp
+    ost = OState(ec.budget, ec.root_token)
+    frontier = [0]
+    t = 0.0
     done = 0
-    t_attn = 0.0
-    order = [(b, i) for i in range(T) for b in range(B)]
-    while done < len(order) and t_attn < budget_s:
-        rows = {order[done]}
+    for call in range(min(rounds, len(zs))):
+        z = zs[call].double().numpy()
         t0 = time.perf_counter()
-        o_attn(host["q"], host["k_cache"], host["v_cache"], host["prefix_len"], host["k_tree"],
-               host["v_tree"], host["parent"], sparse_topk=a.sparse_topk, block_size=a.block_size, rows=rows)
-        t_attn += time.perf_counter() - t0
+        frontier = list(expand_call(ost, z[:len(frontier)], np.asarray(frontier, np.int64), ec.Bsel))
+        t += time.perf_counter() - t0
         done += 1
-    per_node = t_attn / done
-    t_step = per_node * B * T + t_acc + t_exp
-    return {"value": (B * T) / t_step, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
-            "sample": f"attention of {done} of {B * T} nodes (all heads, fp64) scaled to the step, "
-                      f"plus the full acceptance walk ({t_acc:.2f} s){exp_note}",
-            "seconds": round(t_attn + t_acc + t_exp, 2)}
+    return t / done * len(zs), done, len(zs)
+
+
+def cpu_baseline(host, budget_s=15.0, runner=None):
+    """The oracle's whole-step throughput on the host cores: a bounded
+    sample of the attention (tasks of (sequence, kv head, nodes) on a spawned
+    process pool, wall-timed and scaled to every (node, kv head)), the full
+    acceptance walk (one task per sequence), and for the SpecExec workload
+    the expansion build (its first rounds, scaled).  Also the 1-worker time
+    of the same work, from one call on one thread."""
+    own = runner is None
+    r = runner or OracleRunner(host)
+    try:
+        per_unit = r.one_worker_node_seconds()
+        wall, units, sample = r.time_attention(budget_s, per_unit)
+        all_units = r.B * r.T * r.Hkv
+        t_attn = wall / units * all_units
+        t_acc, t_acc_1 = r.time_accept(list(range(r.B)))
+        t_exp, exp_note = 0.0, ""
+        if host["exp"] is not None:
+            t_exp, done, n = time_expand_oracle(host["exp"])
+            exp_note = f"; expansion: {done} of {n} rounds timed (sequential), scaled to the build"
+        t_step = t_attn + t_acc + t_exp
+        t_step_1 = per_unit * all_units + t_acc_1 + t_exp
+        tokens = r.B * r.T
+        return {"value": tokens / t_step, "unit": "tokens/s", "cores": r.workers, "kind": "oracle",
+                "workers": r.workers, "value_1worker": tokens / t_step_1,
+                "sample": f"attention of {units} of {all_units} (node, kv head) pairs (fp64, all heads of the "
+                          f"group) on {r.workers} spawned workers of one BLAS thread, wall {wall:.1f} s, scaled to "
+                          f"the step; acceptance of all {r.B} sequences ({t_acc:.2f} s){exp_note}; the 1-worker "
+                          f"value scales one single-thread call ({per_unit:.3f} s per pair)",
+                "seconds": round(wall + t_acc + t_exp, 2)}
+    finally:
+        if own:
+            r.close()
 
 
 # --------------------------------------------------------------------------
@@ -533,34 +880,115 @@ def config_block(step, world):
 
 
 def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step is a bounded sample of the
+    workload on the host cores, scaled to tokens per second."""
     if rank != 0:
         return
-    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
-    step = Step(args.config, 0, dev)
-    vals = []
-    for k in range(args.warmup + args.steps):
-        cb = cpu_baseline(step, budget_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
-        if k >= args.warmup:
-            vals.append(cb)
-    v = statistics.median([x["value"] for x in vals])
+    host = host_inputs(args.config, 0)
+    runner = OracleRunner(host)
+    try:
+        per_unit = runner.one_worker_node_seconds()
+        budget = max(2.0, 45.0 / max(1, args.steps + args.warmup))
+        t_exp = 0.0
+        if host["exp"] is not None:
+            t_exp, _, _ = time_expand_oracle(host["exp"], rounds=1)
+        all_units = runner.B * runner.T * runner.Hkv
+        workers = runner.workers
+        vals = []
+        for k in range(args.warmup + args.steps):
+            wall, units, _ = runner.time_attention(budget, per_unit)
+            b = k % runner.B
+            _, t_one = runner.time_accept([b])
+            t_acc = t_one * -(-runner.B // workers)
+            t_step = wall / units * all_units + t_acc + t_exp
+            if k >= args.warmup:
+                vals.append(runner.B * runner.T / t_step)
+        v = statistics.median(vals)
+    finally:
+        runner.close()
+    from synth import CONFIGS
+    base = "longctx" if args.config == "longctx_sparse" else args.config
+    shim = type("S", (), dict(c=CONFIGS[base], name=args.config, temperature=host["temp"],
+                              sparse=args.config == "longctx_sparse", B=runner.B, T=runner.T))()
+    sample = (f"per step: attention of a bounded sample of (sequence, kv head, node) tasks on {workers} "
+              f"spawned workers (about {budget:.0f} s), one sequence's acceptance walk (the pool walks "
+              f"{min(workers, runner.B)} sequences at once), scaled to the step"
+              + ("; expansion: one round timed, scaled to the build" if host["exp"] is not None else ""))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * step.B * step.T / v,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * runner.B * runner.T / v,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_block(step, 1),
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"], "kind": "oracle",
-                             "sample": vals[0]["sample"]},
+            "data": "synthetic", "config": config_block(shim, 1),
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": workers, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def main_roofline(step, ms, hbm, bf16, src):
+    """The roofline object of the step's dominant call."""
+    attn_s, acc_s = ms["attn"] * 1e-3, ms["accept"] * 1e-3
+    exp_s = ms.get("expand", 0.0) * 1e-3
+    if exp_s >= max(acc_s, attn_s):
+        achieved = step.expand_bytes / exp_s / 1e9
+        roof = {"kernel": "tree_expand_topb (16 rounds: row + merge launches)", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                "algorithmic_bytes": step.expand_bytes, "units": "draft logit rows of all rounds x V x 4 B"}
+        tk = "expand_rows_kernel"
+    elif acc_s >= attn_s:
+        achieved = step.accept_bytes / acc_s / 1e9
+        roof = {"kernel": "accept_node_kernel (tree_accept: one launch)", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                "algorithmic_bytes": step.accept_bytes, "units": "B x T x V x 4 B of target logits (+ draft rows)"}
+        tk = "accept_node_kernel"
+    elif step.attn_bytes / (hbm * 1e9) >= step.attn_flops / (bf16 * 1e12):
+        achieved = step.attn_bytes / attn_s / 1e9
+        roof = {"kernel": "tree_verify_attn", "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                "algorithmic_bytes": step.attn_bytes, "units": "every prefix and tree K/V element once"}
+        tk = "attn_tc_kernel"
+    else:
+        achieved = step.attn_flops / attn_s / 1e12
+        roof = {"kernel": "tree_verify_attn", "bound": "tensor", "achieved": round(achieved, 2),
+                "peak": bf16, "unit": "TFLOP/s", "frac": round(achieved / bf16, 4),
+                "algorithmic_flops": step.attn_flops, "units": "4 d Hq x sum over nodes of |K(i)|"}
+        tk = "attn_tc_kernel"
+    roof["peak_source"] = src + " (MEASURED_PEAKS.json: burst figures, each call timed alone)" \
+        if src == "measured" else src
+    # against the 8 TB/s / 2.25 PFLOP/s denominators
+    tpk = TARGET_HBM_GBS if roof["bound"] == "hbm" else TARGET_BF16_TFLOPS
+    roof["frac_target"] = round(roof["achieved"] / tpk, 4)
+    roof["traffic"] = None
+    if tk == "attn_tc_kernel" and step.attn_path == 4:
+        tk = "attn_pair_kernel"
+    if tk in ("attn_tc_kernel", "attn_pair_kernel") and step.attn_path in (1, 4):
+        roof["kernel"] = f"{tk} (tree_verify_attn: one launch)"
+    if tk not in ("attn_tc_kernel", "attn_pair_kernel") or step.attn_path in (1, 4):
+        roof["traffic"] = measured_traffic(tk, step.name)
+        roof["traffic_source"] = "profiles/traffic.txt (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
+    return roof
+
+
+def run_config(name, args, world, rank, dev, flush, K, W, with_e2e):
+    """Build one workload, time its step, and summarise it."""
+    step = Step(name, seed=rank, dev=dev)
+    times = time_steps(step, K, W, world, flush)
+    ms, summary = call_summary(step, times, world)
+    res = {"step": step, "ms": ms, "summary": summary}
+    if with_e2e:
+        e2e_ms, h2d, d2h = time_e2e(step, max(3, K // 5), 3, flush)
+        res["e2e"] = (max_over_ranks(e2e_ms, world), h2d, d2h)
+        commit_ms, commit_bytes = time_commit(step, max(3, K), 3, flush)
+        res["commit"] = (max_over_ranks(commit_ms, world), commit_bytes)
+    return res
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="llama3_8b",
-                    choices=["llama3_8b", "specexec70b", "serving", "longctx", "longctx_sparse", "tiny"])
+    ap.add_argument("--config", default="longctx", choices=CONFIG_NAMES)
+    ap.add_argument("--only", action="store_true", help="time the main workload alone (no other configs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -574,86 +1002,53 @@ def main():
     from tree_verification_verify_b200 import build
     build.build()
     dev = torch.device("cuda", torch.cuda.current_device())
-    step = Step(args.config, seed=rank, dev=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     clk = ClockSampler(local)
     clk.start()
-    times = time_steps(step, args.steps, args.warmup, world, flush)
+    main_res = run_config(args.config, args, world, rank, dev, flush, args.steps, args.warmup, True)
     clocks = clk.stop()
-    ms_step = max_over_ranks(statistics.fmean(times["step"]), world)
-    ms_calls = max_over_ranks(statistics.fmean([sum(ts) for ts in zip(*[times[nm] for nm in times if nm != "step"])]),
-                              world)
-    ms_attn = max_over_ranks(statistics.fmean(times["attn"]), world)
-    ms_acc = max_over_ranks(statistics.fmean(times["accept"]), world)
-    ms_exp = max_over_ranks(statistics.fmean(times["expand"]), world) if "expand" in times else 0.0
-    e2e_ms, h2d, d2h = time_e2e(step, max(3, args.steps // 5), 3, flush)
-    e2e_ms = max_over_ranks(e2e_ms, world)
-    commit_ms, commit_bytes = time_commit(step, max(3, args.steps), 3, flush)
-    commit_ms = max_over_ranks(commit_ms, world)
-    tokens = step.B * step.T * world
+    step, ms, summary = main_res["step"], main_res["ms"], main_res["summary"]
     hbm, bf16, bf16_sus, src = peaks()
-    # dominant call and its roofline
-    attn_t = max(step.attn_bytes / (hbm * 1e9), step.attn_flops / (bf16 * 1e12))
-    if ms_exp >= max(ms_acc, ms_attn):
-        achieved = step.expand_bytes / (ms_exp * 1e-3) / 1e9
-        roof = {"kernel": "tree_expand_topb (16 rounds: row + merge launches)", "bound": "hbm",
-                "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                "traffic": None, "peak_source": src, "algorithmic_bytes": step.expand_bytes}
-        tk = "expand_rows_kernel"
-    elif ms_acc >= ms_attn:
-        achieved = step.accept_bytes / (ms_acc * 1e-3) / 1e9
-        roof = {"kernel": "accept_node_kernel (tree_accept: one launch)", "bound": "hbm",
-                "achieved": round(achieved, 1),
-                "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
-                "peak_source": src, "algorithmic_bytes": step.accept_bytes}
-        tk = "accept_node_kernel"
-    else:
-        if step.attn_bytes / (hbm * 1e9) >= step.attn_flops / (bf16 * 1e12):
-            achieved = step.attn_bytes / (ms_attn * 1e-3) / 1e9
-            roof = {"kernel": "tree_verify_attn (all launches)", "bound": "hbm", "achieved": round(achieved, 1),
-                    "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
-                    "peak_source": src, "algorithmic_bytes": step.attn_bytes}
-            tk = "attn_tc_kernel"
-        else:
-            achieved = step.attn_flops / (ms_attn * 1e-3) / 1e12
-            roof = {"kernel": "tree_verify_attn (all launches)", "bound": "tensor", "achieved": round(achieved, 2),
-                    "peak": bf16, "unit": "TFLOP/s", "frac": round(achieved / bf16, 4), "traffic": None,
-                    "peak_source": src, "algorithmic_flops": step.attn_flops}
-            tk = "attn_tc_kernel"
-    if tk == "attn_tc_kernel" and step.attn_path == 1:
-        roof["kernel"] = "attn_tc_kernel (tree_verify_attn: one launch)"
-    if step.attn_path != 1 and tk == "attn_tc_kernel":
-        roof["kernel"] = "tree_verify_attn (all launches)"
-    else:
-        roof["traffic"] = measured_traffic(tk, step.name)
-        roof["traffic_source"] = "profiles/traffic.txt (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
+    e2e_ms, h2d, d2h = main_res["e2e"]
+    commit_ms, commit_bytes = main_res["commit"]
+    tokens = step.B * step.T * world
     line = {
-        "metric": METRIC, "value": tokens / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "metric": METRIC, "value": tokens / (ms["step"] * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms["step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_block(step, world),
-        "roofline": roof,
-        "calls": {"tree_verify_attn_us": round(ms_attn * 1e3, 2), "tree_accept_us": round(ms_acc * 1e3, 2),
-                  "attn_roofline_frac": round(attn_t / (ms_attn * 1e-3), 4),
-                  "attn_tflops": round(step.attn_flops / (ms_attn * 1e-3) / 1e12, 2),
-                  "accept_gbs": round(step.accept_bytes / (ms_acc * 1e-3) / 1e9, 1),
-                  "accept_nodes_per_s": step.B * step.T / (ms_acc * 1e-3)},
+        "roofline": main_roofline(step, ms, hbm, bf16, src),
+        "calls": summary,
         "launches_per_step": step.launches_per_step(),
-        "ms_per_step_call_by_call": round(ms_calls, 5),
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "note": "every step copies all of its inputs (KV cache included) from pinned host memory"},
         "gpu_launches": step.launches_per_step() * args.steps,
         "clocks": clocks,
+        "near_threshold": step.near_threshold(),
     }
-    # the KV commit of the accepted paths (not part of the timed step)
-    line["calls"]["tree_commit_kv_us"] = round(commit_ms * 1e3, 2)
-    line["calls"]["commit_bytes"] = commit_bytes
-    line["calls"]["commit_gbs"] = round(commit_bytes / (commit_ms * 1e-3) / 1e9, 1)
-    if step.expand:
-        line["calls"]["tree_expand_us"] = round(ms_exp * 1e3, 2)
-        line["calls"]["expand_gbs"] = round(step.expand_bytes / (ms_exp * 1e-3) / 1e9, 1)
+    line["calls"]["tree_commit_kv"] = {"us": round(commit_ms * 1e3, 2), "bytes": commit_bytes,
+                                       "gbs": round(commit_bytes / (commit_ms * 1e-3) / 1e9, 1)}
+    host = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(step)
+        host = host_inputs(args.config, device_step=step)
+    step.free()
+    del main_res
+    if not args.only and args.config == "longctx":
+        line["configs"] = {}
+        clk2 = ClockSampler(local)
+        clk2.start()
+        for name in EXTRA_CONFIGS:
+            r = run_config(name, args, world, rank, dev, flush, max(5, min(args.steps, 10)), 3, False)
+            s = r["summary"]
+            s["workload"] = config_block(r["step"], world)["workload"]
+            s["near_threshold"] = r["step"].near_threshold()
+            line["configs"][name] = s
+            r["step"].free()
+            del r
+        line["configs_clocks"] = clk2.stop()
+    if host is not None:
+        line["cpu_baseline"] = cpu_baseline(host)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
