@@ -122,7 +122,7 @@ def select_blocks(qi_group, kbar_bg, nblk, topk):
 
 def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent,
                      n_nodes=None, scale=0.0, sparse_topk=0, block_size=64,
-                     k_block_mean=None, rows=None):
+                     k_block_mean=None, rows=None, forced_sel=None):
     """Oracle for tree_verify_attn.
 
     Shapes: q [B][T][Hq][d], k_cache/v_cache [B][Lmax][Hkv][d],
@@ -135,7 +135,11 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent,
     sel_gap [B][T][Hkv] relative rank-k/k+1 score gap (sparse only),
     status (int bit set).  `rows`, a set of (b, i) pairs, restricts the
     computation to those nodes (sampled checks of large cases); the status
-    word is still computed over every node.
+    word is still computed over every node.  `forced_sel` [B][T][Hkv][k]
+    (block ids, -1 ignored), sparse only: the node attends to these blocks
+    instead of its own top-k (sel and sel_gap still report the top-k); this
+    checks an output whose selection was taken elsewhere at a near-tie of
+    the k-th and (k+1)-th block scores.
     """
     Q = _f64(q)
     K = _f64(k_cache)
@@ -193,6 +197,8 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent,
                     kept, gap, _ = select_blocks(Q[b, i, g * G:(g + 1) * G], kbar[b, :nblk, g], nblk, topk)
                     sel[b, i, g, :len(kept)] = kept
                     sel_gap[b, i, g] = gap
+                    if forced_sel is not None:
+                        kept = sorted(int(j) for j in np.asarray(forced_sel[b][i][g]) if 0 <= j < nblk)
                     pos = [p for j in kept for p in range(j * block_size, min((j + 1) * block_size, Lb))]
                     kp = K[b, pos, g]
                     vp = Vc[b, pos, g]

@@ -57,14 +57,19 @@ def check_attn(gpu_out, ref, dtype, lse_gpu=None, rows_mask=None, poison=None):
     return max_abs, rel
 
 
-def check_accept(gpu, ref, parent, T):
+def check_accept(gpu, ref, parent, T, V=None, draft_tokens=None, what=""):
     """Exact comparison of acceptance outputs per sequence; sequences whose
     oracle walk met a decision within NEAR of its threshold are only
-    checked for validity.  Returns (exact, near)."""
+    checked for validity (a root path of the tree, the path's draft tokens
+    emitted in order, a bonus token in [0, V)).  Prints and returns
+    (exact, near); callers bound `near`."""
     n_acc = gpu["n_accepted"].cpu().numpy()
     acc = gpu["accepted_nodes"].cpu().numpy()
     tok = gpu["out_tokens"].cpu().numpy()
     par = parent.cpu().numpy() if isinstance(parent, torch.Tensor) else np.asarray(parent)
+    dtok = None
+    if draft_tokens is not None:
+        dtok = draft_tokens.cpu().numpy() if isinstance(draft_tokens, torch.Tensor) else np.asarray(draft_tokens)
     exact = near = 0
     for b in range(len(n_acc)):
         if ref["min_margin"][b] < NEAR:
@@ -76,9 +81,22 @@ def check_accept(gpu, ref, parent, T):
                 assert par[b, j] == c
                 c = int(j)
             assert np.all(acc[b, k:] == -1)
+            if dtok is not None:
+                np.testing.assert_array_equal(tok[b, :k], dtok[b, acc[b, :k]])
+            if V is not None:
+                assert 0 <= tok[b, k] < V, (b, tok[b, k])
+            assert np.all(tok[b, k + 1:] == -1)
             continue
         exact += 1
         assert int(n_acc[b]) == int(ref["n_accepted"][b]), (b, n_acc[b], ref["n_accepted"][b])
         np.testing.assert_array_equal(acc[b], ref["accepted_nodes"][b])
         np.testing.assert_array_equal(tok[b], ref["out_tokens"][b])
+    print(f"acceptance parity {what}: {exact} sequences exact, {near} near-threshold (|margin| < {NEAR})")
     return exact, near
+
+
+def near_allowed(B):
+    """Near-threshold sequences a parity case may contain: at most 1% of its
+    sequences (none below 100 sequences; every fixed-seed case here has
+    none in the oracle)."""
+    return B // 100

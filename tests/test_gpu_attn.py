@@ -12,7 +12,7 @@ import torch
 from oracle.attention import tree_verify_attn as oracle_attn, ST_BAD_PARENT, ST_BAD_LEN
 from synth import (attn_case, config_attn_case, tree_binary, tree_chain, tree_star,
                    tree_bfs_fanout, tree_random_recursive, tree_random_depth_limited, CONFIGS)
-from parity_util import check_attn, cuda
+from parity_util import check_attn, cuda, BF16_MAX_ABS, BF16_REL_L2, FP32_MAX_ABS, FP32_REL_L2
 
 pytestmark = pytest.mark.gpu
 POISON = 512.0          # exactly representable in bf16 and fp32
@@ -74,6 +74,9 @@ SHAPES = [
     (1, 600, 64, 8, 128, [5000], "bf16", "recursive"),   # split prefix + cluster merge
     (1, 300, 32, 8, 128, [2000], "bf16", "chain"),       # ragged last row tile after 3 tree tiles
     (1, 1000, 64, 8, 128, [300], "bf16", "chain"),       # 8 tree tiles per row tile
+    (1, 256, 32, 8, 128, [20000], "bf16", "bfs"),        # long prefix (two-tile CTAs where the plan picks them)
+    (2, 100, 16, 2, 128, [9000, 3000], "bf16", "recursive"),  # odd tile count: a last pair with one tile
+    (1, 200, 8, 8, 128, [12000], "bf16", "chain"),       # G = 1: 128 nodes per tile, deep tree tiles
 ]
 
 
@@ -88,8 +91,8 @@ def test_shapes(shape):
     o, lse, _, st = _gpu(case)
     import tree_verification_verify_b200 as tv
     # bf16 with d = 128 and a power-of-two group runs the tensor-core kernel
-    assert tv.last_attn_path == (1 if (dtype == "bf16" and d == 128) else 0)
-    assert tv.last_attn_launches == (1 if tv.last_attn_path == 1 else 3)
+    assert tv.last_attn_path in ((1, 4) if (dtype == "bf16" and d == 128) else (0,))
+    assert tv.last_attn_launches == (1 if tv.last_attn_path in (1, 4) else 3)
     ref = _oracle(case)
     check_attn(o, ref, o.dtype, lse_gpu=lse, poison=POISON)
     assert st == ref["status"] == 0
@@ -148,7 +151,7 @@ def test_full_size_dense_sampled(name, per_b):
     case = config_attn_case(name, seed=0)
     o, lse, _, st = _gpu(case)
     import tree_verification_verify_b200 as tv
-    assert tv.last_attn_path == 1
+    assert tv.last_attn_path in (1, 4)
     rows = _sample_rows(c["B"], c["T"], per_b, 1)
     ref = _oracle(case, rows=rows)
     check_attn(o, ref, torch.bfloat16, lse_gpu=lse, rows_mask=_rows_mask(rows, c["B"], c["T"]))
@@ -166,25 +169,62 @@ def test_sparse_small_all_blocks_equals_dense():
     assert (od.float() - os_.float()).abs().max().item() < 2e-2
 
 
+# Block selection band.  The GPU scores a block as <sum_h q_h, kbar_j> in
+# fp32: kbar from 64 bf16 keys and the group sum of G bf16 queries are exact
+# or within one fp32 rounding, and the d-term dot product carries at most
+# about d * 2^-24 * sum_i |a_i b_i| of rounding.  On these inputs sum |a_i b_i|
+# stays within a few times max |score|, so two scores closer than about
+# 1e-6 of max |score| can swap; SPARSE_BAND is that bound with a margin of
+# ten.  Where the GPU's kept set differs from the oracle's, the oracle's
+# rank-k / rank-(k+1) gap must lie inside the band, such pairs may be at
+# most 1% of the checked (node, kv head) pairs, and their output is checked
+# against the oracle run with the GPU's own selection.
+SPARSE_BAND = 1e-5
+
+
 def _check_sparse(case, rows, B, T, Hkv, G, k):
     o, lse, sel, st = _gpu(case, want_sel=True)
     ref = _oracle(case, rows=rows)
     sel = sel.cpu().numpy()
-    checked = near = 0
-    for (b, i) in rows:
+    got = o.double().cpu().numpy()
+    lg = lse.double().cpu().numpy()
+    bf16 = o.dtype == torch.bfloat16
+    same, near = [], []
+    for (b, i) in sorted(rows):
         for g in range(Hkv):
-            if not np.array_equal(sel[b, i, g], ref["sel"][b, i, g]):
-                # only an fp32 near-tie at the k-th block may differ
-                assert ref["sel_gap"][b, i, g] < 1e-4, (b, i, g, ref["sel_gap"][b, i, g])
-                near += 1
-                continue
-            hs = slice(g * G, (g + 1) * G)
-            got = o[b, i, hs].double().cpu().numpy()
-            want = ref["out"][b, i, hs]
-            assert np.max(np.abs(got - want)) <= 2e-2
-            checked += 1
-    assert checked > 0
-    return checked, near, st
+            if np.array_equal(sel[b, i, g], ref["sel"][b, i, g]):
+                same.append((b, i, g))
+            else:
+                assert ref["sel_gap"][b, i, g] < SPARSE_BAND, (b, i, g, ref["sel_gap"][b, i, g])
+                near.append((b, i, g))
+    pairs = len(rows) * Hkv
+    print(f"block selection: {len(same)} of {pairs} (node, kv head) pairs equal to the oracle's, "
+          f"{len(near)} near-ties inside the band")
+    assert len(near) <= max(1, pairs // 100)
+
+    def compare(items, want_out, want_lse):
+        g_ = np.concatenate([got[b, i, g * G:(g + 1) * G].ravel() for b, i, g in items])
+        w_ = np.concatenate([want_out[b, i, g * G:(g + 1) * G].ravel() for b, i, g in items])
+        d = g_ - w_
+        max_abs = float(np.max(np.abs(d)))
+        rel = float(np.linalg.norm(d) / max(np.linalg.norm(w_), 1e-300))
+        if bf16:
+            assert max_abs <= BF16_MAX_ABS and rel <= BF16_REL_L2, (max_abs, rel)
+        else:
+            assert max_abs <= FP32_MAX_ABS and rel <= FP32_REL_L2, (max_abs, rel)
+        dl = max(float(np.max(np.abs(lg[b, i, g * G:(g + 1) * G] - want_lse[b, i, g * G:(g + 1) * G])))
+                 for b, i, g in items)
+        assert dl <= (2e-3 if bf16 else 2e-5), dl
+        return max_abs, rel
+
+    assert same
+    compare(same, ref["out"], ref["lse"])
+    if near:
+        ref2 = oracle_attn(case.q, case.k_cache, case.v_cache, case.prefix_len, case.k_tree, case.v_tree,
+                           case.parent, n_nodes=case.n_nodes, scale=case.scale, sparse_topk=case.sparse_topk,
+                           block_size=case.block_size, rows={(b, i) for b, i, _ in near}, forced_sel=sel)
+        compare(near, ref2["out"], ref2["lse"])
+    return len(same), len(near), st
 
 
 def test_sparse_small_offsets():
@@ -217,7 +257,7 @@ def test_sparse_shapes(Hq, Hkv, d, dtype, bs, k):
 def test_full_size_sparse_sampled():
     c = CONFIGS["longctx"]
     case = config_attn_case("longctx", seed=0, sparse=True)
-    rows = _sample_rows(c["B"], c["T"], 3, 2)
+    rows = _sample_rows(c["B"], c["T"], 64, 2)          # 64 sampled nodes per sequence, plus the first and last
     checked, near, st = _check_sparse(case, rows, c["B"], c["T"], c["Hkv"], c["Hq"] // c["Hkv"], 32)
     assert st == 0
     import tree_verification_verify_b200 as tv

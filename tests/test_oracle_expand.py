@@ -231,3 +231,29 @@ def test_specexec_sized_invariants():
     for r in range(16):
         lo, hi = 1 + r * Bsel, min(1 + (r + 1) * Bsel, budget)
         assert np.all(np.diff(lp[lo:hi]) <= 0)
+
+
+def test_nonfinite_row_consumes_its_node():
+    """A row holding a non-finite logit adds no candidates, sets the
+    NONFINITE bit, and still counts as the node's expansion: the same node
+    given again is a bad row.  Rows given alongside it expand normally."""
+    from oracle.attention import ST_NONFINITE, ST_BAD_ROW
+    st = ExpandState(16)
+    z = np.zeros((1, 4))
+    z[0, 2] = np.inf
+    new = expand_call(st, z, [0], 2)
+    assert new == [] and st.n_nodes == 1
+    assert st.status & ST_NONFINITE and not st.status & ST_BAD_ROW
+    assert 0 in st.expanded
+    new = expand_call(st, np.zeros((1, 4)), [0], 2)
+    assert new == [] and st.status & ST_BAD_ROW
+    # a NaN row next to a finite one: the NaN row's node gets no children
+    # (the pool still holds the root's third child), the finite one does
+    st = ExpandState(16)
+    new = expand_call(st, np.array([[0.0, 1.0, 2.0]]), [0], 2)          # nodes 1, 2 (tokens 2, 1)
+    z = np.array([[np.nan, 0.0, 0.0], [5.0, 0.0, 0.0]])
+    new = expand_call(st, z, new, 3)
+    assert st.status & ST_NONFINITE
+    parents = [st.parent[i] for i in new]
+    assert 1 not in parents and 2 in parents
+    assert 1 in st.expanded and 2 in st.expanded

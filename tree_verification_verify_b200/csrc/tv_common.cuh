@@ -63,9 +63,12 @@ constexpr int kTagSpecExec = 3;
 
 // ---------------------------------------------------------------- keys
 // Order-preserving maps: a < b  <=>  key(a) < key(b) (for non-NaN input).
+// -0.0 and +0.0 compare equal, so they get one key (that of +0.0): equal
+// values must tie and fall to the index tie-break.
 
 __device__ __forceinline__ uint32_t f32_key(float x) {
-  const uint32_t u = __float_as_uint(x);
+  uint32_t u = __float_as_uint(x);
+  u = (u == 0x80000000u) ? 0u : u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 __device__ __forceinline__ float key_f32(uint32_t k) {
@@ -73,7 +76,8 @@ __device__ __forceinline__ float key_f32(uint32_t k) {
   return __uint_as_float(u);
 }
 __device__ __forceinline__ uint64_t f64_key(double x) {
-  const uint64_t u = static_cast<uint64_t>(__double_as_longlong(x));
+  uint64_t u = static_cast<uint64_t>(__double_as_longlong(x));
+  u = (u == 0x8000000000000000ull) ? 0ull : u;
   return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
 __device__ __forceinline__ double key_f64(uint64_t k) {
