@@ -344,11 +344,14 @@ TV_API tv_status tree_commit_kv(const tv_commit_args* a, tv_stream_t stream);
  * 0 = CUDA-core split-KV, 1 = tcgen05 tensor-core prefix kernel,
  * 2 = block top-k sparse path on CUDA cores, 3 = block top-k sparse path on
  * the tensor-core kernel (bf16, d = 128, blocks of 64, G >= 4),
+ * 4 = the tcgen05 kernel in its two-query-tile form (each CTA takes two
+ * 128-row tiles of packed (node, head) rows that share every K/V tile;
+ * chosen by the same cost model as 1, for long prefixes),
  * -1 = the arguments are rejected. */
 TV_API int32_t tv_attn_path(const tv_attn_args* a);
 /* How many kernels tree_verify_attn launches for these arguments (0 when
  * B or T is 0, -1 when the arguments are rejected): 1 for the tensor-core
- * kernel (its prefix chunks are merged inside the launch), 3 on the
+ * kernels (paths 1 and 4: prefix chunks are merged inside the launch), 3 on the
  * CUDA-core path (prefix, tree paths, merge), 5 or 6 on
  * the block top-k CUDA-core path (block means unless the caller passes
  * them, block scores, block selection, sparse prefix, tree paths, merge),

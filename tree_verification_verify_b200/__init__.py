@@ -250,7 +250,7 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent, n_
 last_attn_path = None
 last_attn_launches = None
 ATTN_PATHS = {0: "cuda-core split-KV", 1: "tcgen05 prefix", 2: "block top-k sparse (cuda cores)",
-              3: "block top-k sparse (tcgen05)"}
+              3: "block top-k sparse (tcgen05)", 4: "tcgen05 prefix, two query tiles per CTA"}
 
 
 # --------------------------------------------------------------- KV commit

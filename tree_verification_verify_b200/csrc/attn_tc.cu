@@ -17,24 +17,29 @@
 // log-sum-exp over distributed shared memory to the CTA of the cluster that
 // merges them; each CTA merges a share of the rows and writes the output.
 //
-// Warp roles (256 threads):
-//   warps 0-3  softmax / correction / epilogue: thread t owns query row t,
-//              which is TMEM lane t (tcgen05.ld 32x32b);
-//   warp 4     Q and the K tiles: TMA into a three-stage ring (128B swizzle,
+// Warp roles (384 threads):
+//   warps 0-7  softmax / correction / epilogue: warps w and w + 4 own TMEM
+//              lanes 32 (w % 4) .. (query rows), warp w < 4 key columns
+//              0-63 of every tile, warp w + 4 columns 64-127 (tcgen05.ld
+//              32x32b).  The two column halves of a row keep independent
+//              online-softmax states, each with its own O accumulator, and
+//              combine them once at the end;
+//   warp 8     Q and the K tiles: TMA into a three-stage ring (128B swizzle,
 //              K-major) or, for tree tiles, a cp.async gather;
-//   warp 5     TMEM allocator and MMA issuer (one thread): S = Q K^T into
-//              one of two TMEM S buffers, O += P V with P read from TMEM;
-//   warp 6     the V tiles, a two-stage ring (MN-major), like warp 4;
-//   warp 7     tree bookkeeping (last chunk): parent[] into shared memory,
+//   warp 9     TMEM allocator and MMA issuer (one thread): S = Q K^T into
+//              one of two TMEM S buffers, O_h += P_h V_h per column half h
+//              with P_h read from TMEM;
+//   warp 10    the V tiles, a two-stage ring (MN-major), like warp 8;
+//   warp 11    tree bookkeeping (last chunk): parent[] into shared memory,
 //              the node bitmap of U, the slot of every node of U and the
 //              slot of its parent.
 // A K stage is released when its S = Q K^T completes, a V stage when its
 // P V completes, so the loads of later tiles start while earlier tiles are
-// in the softmax.  Online softmax in base 2 with a lazily updated row
-// maximum: O and the row sum are rescaled only when the maximum grows by
-// more than 2^8, which keeps P <= 256 (exact in the final O / l).  P is
-// written as bf16 over the first 64 columns of its S buffer.
-//
+// in the softmax.  Online softmax in base 2 with a lazily updated maximum
+// per row half: O_h and its row sum are rescaled only when the half's
+// maximum grows by more than 2^8, which keeps P <= 256 (exact in the final
+// O / l).  P_h is written as bf16 over the first 32 columns of the half's
+// own 64 S columns, so neither half writes where the other still reads.
 // Every mbarrier wait is bounded: on expiry the CTA records TV_DEV_TIMEOUT,
 // stops issuing work, drains what it issued, frees its TMEM, and its rows
 // come out as NaN.
@@ -43,6 +48,7 @@
 #include <cooperative_groups.h>
 
 #include "attn.cuh"
+#include "tc_prims.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -80,9 +86,7 @@ constexpr uint32_t kSmemInbox = kSmemK;                   // merge: fp32 O rows 
 constexpr uint32_t kSmemStage = kSmemV;                   // merge: this CTA's fp32 O rows (idle V ring)
 constexpr int kMaxInboxRows = 144;                        // max over C of C * per (per = 4 * ceil(128 / 4C))
 constexpr uint32_t kTmemCols = 512;                       // S0, S1, O (128 each)
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
-constexpr uint32_t kWaitLimit = 1u << 22;
-constexpr uint32_t kDrainLimit = 1u << 20;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;  // O_h: column half h
 constexpr uint16_t kRootMark = 0xFFFEu;   // parent[] entry of a well-formed root
 constexpr uint16_t kBadMark = 0xFFFFu;    // malformed parent (or no parent slot)
 
@@ -94,7 +98,7 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[kKS], k_empty[kKS];
   uint64_t v_full[kVS], v_empty[kVS];
-  uint64_t s_full[2], p_full[2];
+  uint64_t s_full[2], p_full[2][2];   // p_full[S buffer][column half]
   uint64_t pv_done;
   uint64_t tree_info;
   uint64_t sparse_info;             // block top-k: the union of kept blocks is listed
@@ -107,182 +111,12 @@ struct Bars {
   int node_ok[kRows];               // root path of the tile's node is well formed
   uint64_t inbox_full;              // the cluster's copies into this CTA's inbox have landed
   alignas(16) float st_lse[kRows];  // this CTA's rows: log2-sum-exp (NaN: invalid)
-  uint64_t max_ready[2];            // both halves of every row have posted their tile maximum
-  uint64_t sum_ready;               // both halves have posted their row sums
-  float red_max[2][2][kRows];       // [tile parity][half][row] partial maxima
-  float red_l[2][kRows];            // [half][row] partial row sums
+  uint64_t sum_ready;               // both halves have posted their final maximum and row sum
+  float red_m[2][kRows];            // [half][row] the half's running maximum (log2 units)
+  float red_l[2][kRows];            // [half][row] the half's row sum
   alignas(16) float in_lse[kMaxInboxRows];  // merge inbox: log2-sum-exp of row (chunk, row)
 };
 
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-// Bounded wait on phase `parity`; false when the CTA aborted or the limit
-// expired (then the abort flag is raised).
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort) {
-  const uint32_t a = smem_u32(b);
-  for (uint32_t it = 0; it < kWaitLimit; ++it) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (ok) return true;
-    if ((it & 255u) == 255u && *abort) return false;
-  }
-  *abort = 1;
-  return false;
-}
-
-__device__ __forceinline__ void tma_load_4d(const CUtensorMap* map, uint32_t dst, uint64_t* bar,
-                                            int x, int y, int z, int w) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Shared-memory matrix descriptor: 128B swizzle, version 1 (sm_100).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
-         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) |
-         (1ull << 46) | (2ull << 61);
-}
-
-// Instruction descriptor of kind::f16: bf16 x bf16 -> f32, M x N.
-__host__ __device__ constexpr uint32_t instr_desc(int M, int N, int a_mn_major, int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn_major) << 15) |
-         (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
-         (static_cast<uint32_t>(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
-        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
-        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
-      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
-      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-      : "memory");
-}
-
-// D (TMEM) (+)= A (TMEM, K-major: row m in lane m, two bf16 per column) x B
-// (shared memory descriptor).
-__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Wait used while draining after an abort: bounded, ignores the abort flag.
-__device__ __forceinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
-  const uint32_t a = smem_u32(b);
-  for (uint32_t it = 0; it < kDrainLimit; ++it) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (ok) return;
-  }
-}
 
 // Slot of node a in U: the number of marked nodes below a.
 __device__ __forceinline__ int u_slot(const Bars& bars, int a) {
@@ -291,42 +125,10 @@ __device__ __forceinline__ int u_slot(const Bars& bars, int a) {
 
 __device__ __forceinline__ uint32_t s_col(int j) { return (j & 1) ? kColS1 : kColS0; }
 
-// Shared-memory address `a` of this CTA mapped to CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t cluster_addr(uint32_t a, int rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-  return r;
-}
-
-// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to
-// a cluster peer's, completing on the peer's mbarrier `bar`.
-__device__ __forceinline__ void bulk_s2c(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
-
 // Bytes a merging CTA receives from one chunk for `rows` rows: the fp32 O
 // rows and their log-sum-exp (padded to 16 bytes).
 __host__ __device__ constexpr uint32_t merge_bytes(int rows) {
   return rows > 0 ? static_cast<uint32_t>(rows) * kD * 4 + static_cast<uint32_t>((rows + 3) & ~3) * 4 : 0u;
-}
-
-// Bounded wait (cluster-scope acquire) on phase `parity`; false on expiry.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* b, uint32_t parity) {
-  const uint32_t a = smem_u32(b);
-  for (uint32_t it = 0; it < kWaitLimit; ++it) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (ok) return true;
-  }
-  return false;
 }
 
 }  // namespace tc
@@ -400,8 +202,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     for (int s = 0; s < kVS; ++s) { mbar_init(&bars.v_full[s], 1); mbar_init(&bars.v_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.s_full[s], 1);
-      mbar_init(&bars.p_full[s], kSoftmaxThreads / 32);
-      mbar_init(&bars.max_ready[s], kSoftmaxThreads / 32);
+      mbar_init(&bars.p_full[s][0], kSoftmaxThreads / 64);
+      mbar_init(&bars.p_full[s][1], kSoftmaxThreads / 64);
     }
     mbar_init(&bars.sum_ready, kSoftmaxThreads / 32);
     mbar_init(&bars.pv_done, 1);
@@ -669,18 +471,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       for (int j = 0; ok; ++j) {
         ok = know(j);
         if (!ok || j >= ntot) break;
-        ok = mbar_wait(&bars.p_full[j & 1], (j >> 1) & 1, abort);
-        if (ok) ok = mbar_wait(&bars.v_full[j % kVS], (j / kVS) & 1, abort);
-        if (!ok) break;
-        fence_after();
+        ok = mbar_wait(&bars.v_full[j % kVS], (j / kVS) & 1, abort);
         const uint32_t sv = base + kSmemV + (j % kVS) * kTileBytes;
+        // O_h += P_h V_h: P_h (128 rows x 64 keys, bf16 pairs) sits in the
+        // first 32 columns of the half's own S columns 64 h ..; V_h is rows
+        // 64 h .. 64 h + 63 of the V tile (16 keys = 2 KB per K step).  Once
+        // any of it is issued, its completion is committed (V stage, pv_done)
+        // even when the second half never comes.
+        bool any = false;
+        for (int h = 0; h < 2 && ok; ++h) {
+          ok = mbar_wait(&bars.p_full[j & 1][h], (j >> 1) & 1, abort);
+          if (!ok) break;
+          fence_after();
+          const uint32_t od = tmem + (h ? kColO1 : kColO0);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + kColO, tmem + s_col(j) + kk * 8, smem_desc(sv + kk * 2048, kHalfBytes, 1024),
-                      idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars.v_empty[j % kVS]);
-        mma_commit(&bars.pv_done);
-        ++pv_issued;
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(od, tmem + s_col(j) + 64 * h + kk * 8,
+                        smem_desc(sv + (4 * h + kk) * 2048, kHalfBytes, 1024), idesc_pv,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          any = true;
+        }
+        if (any) {
+          mma_commit(&bars.v_empty[j % kVS]);
+          mma_commit(&bars.pv_done);
+          ++pv_issued;
+        }
+        if (!ok) break;
         const int jn = j + 2;
         ok = know(jn);
         if (!ok) break;
@@ -706,11 +522,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     // ------------------------------------------------------------ softmax warps 0-7
     // Row r is TMEM lane r: warps w and w + 4 share lanes 32 (w % 4) ..; warp
     // w < 4 takes key columns 0-63 of every tile, warp w + 4 columns 64-127.
-    // The two halves exchange their tile maxima (shared memory + mbarrier),
-    // keep their own row sums, and add them at the end.
+    // Each half runs its own online softmax (maximum, row sum, O_h); the two
+    // are combined once, in the epilogue.
     const float sl2 = p.scale * 1.4426950408889634f;   // scores in log2 units
     const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t hcol = 64u * static_cast<uint32_t>(half);
+    const uint32_t ocol = half ? kColO1 : kColO0;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     if (SPARSE) {
@@ -736,12 +553,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       if (j >= ntot) break;
       const bool tree_tile = j >= nprefix;
       const int nk = (tree_tile || SPARSE) ? 0 : min(kKeys, k1 - (k0 + j * kKeys));
+      // a full prefix tile needs no mask (the common case)
+      const bool full = !tree_tile && !SPARSE && nk == kKeys;
       // key mask of this half's 64 columns: two words, kept in registers
-      uint32_t mkA = 0u, mkB = 0u;
+      uint32_t mkA = 0xffffffffu, mkB = 0xffffffffu;
       if (tree_tile) {
         // ancestors of this row's node in slots [128 tt + 64 half, + 64);
         // the tiles run downwards and slots decrease along the path, so the
         // walk continues where the previous tile left it
+        mkA = mkB = 0u;
         const int lo = (ntree - 1 - (j - nprefix)) * kKeys;
         while (cur >= lo) {
           const int w = (cur - lo) >> 5;           // 0..3 in the tile
@@ -766,7 +586,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         const int nh = member ? blk_keys(blk) : 0;
         mkA = nh >= 32 ? 0xffffffffu : (nh <= 0 ? 0u : ((1u << nh) - 1u));
         mkB = nh >= 64 ? 0xffffffffu : (nh <= 32 ? 0u : ((1u << (nh - 32)) - 1u));
-      } else {
+      } else if (!full) {
         const int nh = nk - 64 * half;              // valid keys in this half
         mkA = nh >= 32 ? 0xffffffffu : (nh <= 0 ? 0u : ((1u << nh) - 1u));
         mkB = nh >= 64 ? 0xffffffffu : (nh <= 32 ? 0u : ((1u << (nh - 32)) - 1u));
@@ -779,63 +599,61 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       tmem_ld32(trow + scol + hcol, s);
       tmem_ld32(trow + scol + hcol + 32, s + 32);
       tmem_wait_ld();
-      // masked scores in log2 units; this half's maximum over four
-      // interleaved partial maxima (the maximum does not depend on order)
+      // the half's tile maximum of the raw scores (scale > 0 keeps the
+      // order), over four interleaved partial maxima
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (full) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const uint32_t mw = (c < 32) ? mkA : mkB;
-        s[c] = ((mw >> (c & 31)) & 1u) ? s[c] * sl2 : -INFINITY;
-        mx[c & 3] = fmaxf(mx[c & 3], s[c]);
+        for (int c = 0; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], s[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const uint32_t mw = (c < 32) ? mkA : mkB;
+          s[c] = ((mw >> (c & 31)) & 1u) ? s[c] : -INFINITY;
+          mx[c & 3] = fmaxf(mx[c & 3], s[c]);
+        }
       }
-      const float mh = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      bars.red_max[j & 1][half][row] = mh;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.max_ready[j & 1]);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars.max_ready[j & 1], (j >> 1) & 1, abort));
-      if (!ok) break;
-      const float mt = fmaxf(mh, bars.red_max[j & 1][half ^ 1][row]);
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
       const float m_new = fmaxf(m_run, mt);
-      const bool first = (j == 0);
-      const bool grow = !first && (m_new > m_run + 8.0f);
+      const bool grow = m_new > m_run + 8.0f;       // also the first finite maximum
       float factor = 1.f;
-      if (first) {
-        m_run = m_new;
-      } else if (grow) {
-        factor = ex2_approx(m_run - m_new);
+      if (grow) {
+        factor = ex2_approx(m_run - m_new);         // 0 when m_run = -inf
         m_run = m_new;
       }
-      const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+      const float nmu = (m_run == -INFINITY) ? 0.f : -m_run;
+      // p = 2^(s sl2 - m): one FFMA and one ex2 per score (masked scores are
+      // -inf and give 0)
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        s[c] = ex2_approx(s[c] - mu);
+        s[c] = ex2_approx(fmaf(s[c], sl2, nmu));
         ps[c & 3] += s[c];
       }
       l_run = l_run * factor + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-      if (__any_sync(0xffffffffu, grow)) {
-        // O holds the tiles up to j - 1: wait for their P V, then rescale
-        // this half's 64 columns of O
+      if (__any_sync(0xffffffffu, grow) && j > 0) {
+        // O_h holds the tiles up to j - 1: wait for their P V, then rescale
+        // this half's accumulator (all 128 columns)
         ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (j - 1) & 1, abort));
         if (!ok) break;
         fence_after();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
           float o[32];
-          tmem_ld32(trow + kColO + hcol + c * 32, o);
+          tmem_ld32(trow + ocol + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= factor;
-          tmem_st32(trow + kColO + hcol + c * 32, o);
+          tmem_st32(trow + ocol + c * 32, o);
         }
       }
-      // P as bf16 pairs over the first 64 columns of the S buffer: this
-      // half's keys 64 half .. 64 half + 63 are columns 32 half .. + 31
+      // P_h as bf16 pairs over the first 32 of the half's own 64 S columns
+      // (this thread has read them all already)
       {
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(s[2 * e], s[2 * e + 1]);
-        tmem_st32u(trow + scol + 32u * static_cast<uint32_t>(half), pk);
+        tmem_st32u(trow + scol + hcol, pk);
       }
       tmem_wait_st();
       // V rows that are not keys of this tile (past the prefix end, or an
@@ -846,21 +664,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       if (ragged) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bars.v_full[j % kVS], (j / kVS) & 1, abort));
         if (!ok) break;
-        const bool dead_row = SPARSE ? (row < 64 ? row >= vka : row - 64 >= vkb) : row >= nk;
-        if (half == 0 && dead_row) {
+        // the V rows a half multiplies are its own keys' rows: each half
+        // zeroes the dead rows among its 64
+        const int vr = 64 * half + (row & 63);
+        const bool dead_row = SPARSE ? (half == 0 ? (row & 63) >= vka : (row & 63) >= vkb) : vr >= nk;
+        if (row < 64 && dead_row) {
           uint8_t* sv = gbase + kSmemV + (j % kVS) * kTileBytes;
           const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            *reinterpret_cast<uint4*>(sv + row * 128 + c * 16) = z;
-            *reinterpret_cast<uint4*>(sv + kHalfBytes + row * 128 + c * 16) = z;
+            *reinterpret_cast<uint4*>(sv + vr * 128 + c * 16) = z;
+            *reinterpret_cast<uint4*>(sv + kHalfBytes + vr * 128 + c * 16) = z;
           }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.p_full[j & 1]);
+      if (lane == 0) mbar_arrive(&bars.p_full[j & 1][half]);
     }
     // ------------------------------------------------------------ epilogue
     // The last P V is pv_done's phase ntot - 1.  S(ntot - 1) having landed
@@ -869,33 +690,49 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     if (ok && ntot > 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (ntot - 2) & 1, abort));
     if (ok && ntot > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done, (ntot - 1) & 1, abort));
     fence_after();
-    // the row sum is the two halves' sums
+    // combine the halves: M = max(m_0, m_1), c_h = 2^(m_h - M),
+    // O = (c_0 O_0 + c_1 O_1) / (c_0 l_0 + c_1 l_1); half h writes d columns
+    // 64 h .. 64 h + 63
+    bars.red_m[half][row] = m_run;
     bars.red_l[half][row] = l_run;
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.sum_ready);
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.sum_ready, 0, abort));
-    const float l_row = ok ? l_run + bars.red_l[half ^ 1][row] : 0.f;
+    const float m_o = ok ? bars.red_m[half ^ 1][row] : -INFINITY;
+    const float l_o = ok ? bars.red_l[half ^ 1][row] : 0.f;
+    const float m_0 = half ? m_o : m_run, m_1 = half ? m_run : m_o;
+    const float l_0 = half ? l_o : l_run, l_1 = half ? l_run : l_o;
+    const float M = fmaxf(m_0, m_1);
+    const float c_0 = (m_0 == -INFINITY) ? 0.f : ex2_approx(m_0 - M);
+    const float c_1 = (m_1 == -INFINITY) ? 0.f : ex2_approx(m_1 - M);
+    const float l_row = c_0 * l_0 + c_1 * l_1;
     const bool have = ok && l_row > 0.f;
     const float inv = have ? 1.f / l_row : 0.f;
-    // this half of the row's normalised O into the stage (the idle V ring;
-    // fp32, float4 q of row t at q ^ (t & 7)) and the row's log2-sum-exp
+    const float w0 = c_0 * inv, w1 = c_1 * inv;
+    // this half's columns of the row's normalised O into the stage (the idle
+    // V ring; fp32, float4 q of row t at q ^ (t & 7)) and the row's
+    // log2-sum-exp
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     float* stage = reinterpret_cast<float*>(gbase + kSmemStage) + row * kD;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      float v[32];
-      tmem_ld32(trow + kColO + hcol + c * 32, v);
+      float v0[32], v1[32];
+      tmem_ld32(trow + kColO0 + hcol + c * 32, v0);
+      tmem_ld32(trow + kColO1 + hcol + c * 32, v1);
       tmem_wait_ld();
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const int qq = 16 * half + c * 8 + q;
-        *reinterpret_cast<float4*>(stage + ((qq ^ (row & 7)) * 4)) =
-            have ? make_float4(v[4 * q] * inv, v[4 * q + 1] * inv, v[4 * q + 2] * inv, v[4 * q + 3] * inv)
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 o;
+        o.x = fmaf(w0, v0[4 * q], w1 * v1[4 * q]);
+        o.y = fmaf(w0, v0[4 * q + 1], w1 * v1[4 * q + 1]);
+        o.z = fmaf(w0, v0[4 * q + 2], w1 * v1[4 * q + 2]);
+        o.w = fmaf(w0, v0[4 * q + 3], w1 * v1[4 * q + 3]);
+        *reinterpret_cast<float4*>(stage + ((qq ^ (row & 7)) * 4)) = have ? o : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     const bool good = !(has_tree && !my_ok) && !bad_len && ok;
-    if (half == 0) bars.st_lse[row] = !good ? NAN : (l_row > 0.f ? m_run + __log2f(l_row) : -INFINITY);
+    if (half == 0) bars.st_lse[row] = !good ? NAN : (l_row > 0.f ? M + __log2f(l_row) : -INFINITY);
     // the stage is read by bulk copies (async proxy)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (half == 0 && row_valid && has_tree && !my_ok) set_status(p.status, TV_DEV_BAD_PARENT);
@@ -986,35 +823,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
 
 // ------------------------------------------------------------------ host side
 
+using tcmap::encode_fn;
+using tcmap::make_map;
+
 namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
-  return fn;
-}
-
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
-              int64_t s1, int64_t s2, int64_t s3, uint32_t b1, uint32_t b2) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[4] = {d0, d1, d2, d3};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(s1) * 2, static_cast<cuuint64_t>(s2) * 2,
-                                 static_cast<cuuint64_t>(s3) * 2};
-  const cuuint32_t box[4] = {64, b1, b2, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 bool stride_ok(int64_t s) { return s > 0 && (s * 2) % 16 == 0 && s * 2 < (1ll << 40); }
 

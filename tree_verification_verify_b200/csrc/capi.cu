@@ -16,6 +16,8 @@ cudaError_t launch_expand(const tv_expand_args* a, cudaStream_t stream);
 bool attn_tc_supported(const tv_attn_args* a);
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream);
 int attn_tc_active_clusters(int c);
+cudaError_t launch_attn_pair(const AttnParams& p, cudaStream_t stream);
+int attn_pair_active_clusters(int c);
 bool attn_tc_sparse_supported(const tv_attn_args* a);
 cudaError_t launch_block_means(const AttnParams& p, float* kbar, cudaStream_t stream);
 cudaError_t launch_block_select(const AttnParams& p, cudaStream_t stream);
@@ -41,6 +43,7 @@ bool ws_ok(const void* ws, size_t ws_bytes, size_t need) {
 
 struct AttnPlan {
   bool tc;            // tensor-core prefix kernel
+  bool pair;          // ... in its two-query-tile form (attn_pair.cu)
   bool sparse;
   bool tc_sparse;     // block top-k on the tensor-core kernel
   int nchunk, chunk_len, node_tile, nblk_max;
@@ -64,6 +67,10 @@ tv_status check_attn(const tv_attn_args* a) {
   }
   return TV_OK;
 }
+
+// Time of one 128-key tile in a two-tile CTA (both row tiles), in units of
+// the same tile in a one-tile CTA.
+constexpr double kPairTile = 1.2;
 
 AttnPlan plan_attn(const tv_attn_args* a) {
   AttnPlan pl;
@@ -95,22 +102,29 @@ AttnPlan plan_attn(const tv_attn_args* a) {
     int64_t len = (a->Lmax + want - 1) / want;
     len = (len + 127) / 128 * 128;
     if (pl.tc) {
-      // tensor-core kernel: c chunks of a row tile form one cluster.  Cost
-      // model in tile times: each CTA pays about three tiles of latency
-      // (start-up, first loads, merge) plus its chunk's tiles, and the row
-      // tiles' clusters run in waves of what the device holds at once.
+      // tensor-core kernels: c chunks of a row tile (or of a pair of row
+      // tiles) form one cluster.  Cost model in the time of one 128-key
+      // tile of a one-tile CTA: each CTA pays about three tiles of latency
+      // (start-up, first loads, merge) plus its chunk's tiles, a two-tile
+      // CTA kPairTile per key tile for both of its row tiles, and the
+      // clusters run in waves of what the device holds at once.
       const int64_t tiles = (a->Lmax + 127) / 128;
+      const int64_t units_pair = static_cast<int64_t>(a->B) * a->Hkv * ((ntiles + 1) / 2);
+      const bool pair_ok = a->T <= 2048;
       double best = 1e300;
       int64_t best_len = tiles;
-      for (int c = 1; c <= 8; ++c) {
-        const int64_t lt = (tiles + c - 1) / c;
-        if (c > 1 && lt < 4) break;                       // at least four tiles per chunk
-        if ((tiles + lt - 1) / lt != c) continue;          // c chunks not realisable
-        const int act = attn_tc_active_clusters(c);
-        if (act <= 0) continue;
-        const double waves = static_cast<double>((units + act - 1) / act);
-        const double cost = waves * (3.0 + static_cast<double>(lt));
-        if (cost < best) { best = cost; best_len = lt; }
+      for (int form = 0; form < (pair_ok ? 2 : 1); ++form) {
+        for (int c = 1; c <= 8; ++c) {
+          const int64_t lt = (tiles + c - 1) / c;
+          if (c > 1 && lt < 4) break;                       // at least four tiles per chunk
+          if ((tiles + lt - 1) / lt != c) continue;          // c chunks not realisable
+          const int act = form ? attn_pair_active_clusters(c) : attn_tc_active_clusters(c);
+          if (act <= 0) continue;
+          const int64_t u = form ? units_pair : units;
+          const double waves = static_cast<double>((u + act - 1) / act);
+          const double cost = waves * (3.0 + static_cast<double>(lt) * (form ? kPairTile : 1.0));
+          if (cost < best) { best = cost; best_len = lt; pl.pair = form == 1; }
+        }
       }
       len = best_len * 128;
     }
@@ -152,7 +166,7 @@ extern "C" size_t tree_verify_attn_workspace_size(const tv_attn_args* a) {
 extern "C" int32_t tv_attn_path(const tv_attn_args* a) {
   if (check_attn(a) != TV_OK) return -1;
   const AttnPlan pl = plan_attn(a);
-  return pl.sparse ? (pl.tc_sparse ? 3 : 2) : (pl.tc ? 1 : 0);
+  return pl.sparse ? (pl.tc_sparse ? 3 : 2) : (pl.tc ? (pl.pair ? 4 : 1) : 0);
 }
 
 extern "C" int32_t tv_attn_launches(const tv_attn_args* a) {
@@ -214,7 +228,7 @@ extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws
     e = launch_attn_sparse(p, s);
   } else if (pl.tc) {
     // one kernel: prefix tiles, tree tiles and the cluster merge of the chunks
-    return from_cuda(launch_attn_tc(p, s));
+    return from_cuda(pl.pair ? launch_attn_pair(p, s) : launch_attn_tc(p, s));
   } else {
     e = launch_attn_simt(p, s);
   }
