@@ -443,3 +443,4 @@ def philox_uniforms(seed: int, step: int, b, node, draw, tag, stream=None) -> to
                                     b.data_ptr(), node.data_ptr(), draw.data_ptr(), tag.data_ptr(),
                                     out.data_ptr(), b.numel(), _stream(stream)), "tv_philox_uniforms")
     return out
+

@@ -28,14 +28,14 @@
 //   warps 4-7  the same for tile B;
 //   warp 8     Q (both tiles) and the K tiles: TMA into a two-stage ring
 //              (128B swizzle, K-major) or, for tree tiles, a cp.async gather;
-//   warp 9     TMEM allocator and MMA issuer (one thread);
+//   warp 9     TMEM allocator and MMA issuer (one thread, both tiles);
 //   warp 10    the V tiles, a two-stage ring (MN-major), like warp 8;
 //   warp 11    tree bookkeeping (last chunk): parent[] into shared memory,
 //              the node bitmap of U, the slot of every node of U and the
 //              slot of its parent.
 // A K stage is released when the last S of its tile completes, a V stage
 // when the last P V completes.  S_t(j+1) overwrites P_t(j): it is issued
-// once P_t(j) V has completed.  Online softmax in base 2 with a lazily
+// right behind P_t(j) V (MMAs of one thread execute in issue order).  Online softmax in base 2 with a lazily
 // updated maximum: O_t and its row sum are rescaled only when the maximum
 // grows by more than 2^8, which keeps P <= 256 (exact in the final O / l).
 //
@@ -193,8 +193,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
 
   if (tid == 0) {
     mbar_init(&bars.q_full, 1);
-    for (int s = 0; s < kKS; ++s) { mbar_init(&bars.k_full[s], 1); mbar_init(&bars.k_empty[s], 1); }
-    for (int s = 0; s < kVS; ++s) { mbar_init(&bars.v_full[s], 1); mbar_init(&bars.v_empty[s], 1); }
+    for (int s = 0; s < kKS; ++s) { mbar_init(&bars.k_full[s], 1); mbar_init(&bars.k_empty[s], nq); }
+    for (int s = 0; s < kVS; ++s) { mbar_init(&bars.v_full[s], 1); mbar_init(&bars.v_empty[s], nq); }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars.s_full[t], 1);
       mbar_init(&bars.p_full[t], 4);
@@ -223,6 +223,92 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
   // a softmax thread's row after its main loop: log2-sum-exp (NaN: invalid)
   // and 1 / row sum (0: no keys), staged in the tile's merge round
   float ep_lse2 = NAN, ep_inv = 0.f;
+
+  // ------------------------------------------------------------ MMA issuer
+  // One thread issues both tiles' chains: S_t(0), then per key tile j and
+  // tile t, P_t(j) V and S_t(j + 1), which overwrites P_t(j) in TMEM.  MMAs
+  // issued by one thread execute in issue order, so S_t(j + 1) queued behind
+  // P_t(j) V writes S_t only after that MMA has read P_t(j): both go to the
+  // tensor pipe back to back.  Issuing tile A's pair, then tile B's, keeps
+  // the two softmaxes a half period apart (each runs while the other tile's
+  // MMAs execute); one issuer per tile lets them drift into step and fight
+  // for the same schedulers.  A K or V stage is released when both tiles'
+  // MMAs that read it have completed (the empty barriers count one commit
+  // per tile).
+  auto run_issuer = [&]() {
+    bool ok = true;
+    int ntot = nprefix;
+    bool tree_known = !has_tree;
+    // the tree tiles follow the prefix tiles; their count is known once the
+    // tree warp has built U
+    auto know = [&](int upto) -> bool {
+      if (!tree_known && upto >= nprefix) {
+        if (!mbar_wait(&bars.tree_info, 0, abort)) return false;
+        ntot += (bars.nU + kKeys - 1) / kKeys;
+        tree_known = true;
+      }
+      return true;
+    };
+    const uint32_t idesc_qk = instr_desc(kRows, kKeys, 0, 0);
+    const uint32_t idesc_pv = instr_desc(kRows, kD, 0, 1);
+    int s_issued[2] = {0, 0}, pv_issued[2] = {0, 0};
+    // S_t(j) = Q_t K_j^T into S_t
+    auto issue_s = [&](int t, int j) {
+      const uint32_t sq = base + kSmemQ + t * kTileBytes;
+      const uint32_t sk = base + kSmemK + (j % kKS) * kTileBytes;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+        mma_bf16(tmem + col_s(t), smem_desc(sq + off, 16, 1024), smem_desc(sk + off, 16, 1024), idesc_qk,
+                 kk > 0);
+      }
+      mma_commit(&bars.s_full[t]);
+      mma_commit(&bars.k_empty[j % kKS]);
+      ++s_issued[t];
+    };
+    // O_t += P_t(j) V_j, P_t read from the first 64 columns of S_t
+    auto issue_pv = [&](int t, int j) {
+      const uint32_t sv = base + kSmemV + (j % kVS) * kTileBytes;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, smem_desc(sv + kk * 2048, kHalfBytes, 1024),
+                    idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&bars.pv_done[t]);
+      mma_commit(&bars.v_empty[j % kVS]);
+      ++pv_issued[t];
+    };
+    ok = know(0);
+    if (ok && ntot > 0) ok = mbar_wait3(&bars.q_full, 0, &bars.k_full[0], 0, nullptr, 0u, abort);
+    if (ok && ntot > 0) {
+      fence_after();
+      for (int t = 0; t < nq; ++t) issue_s(t, 0);
+    }
+    for (int j = 0; ok; ++j) {
+      ok = know(j);
+      if (!ok || j >= ntot) break;
+      ok = know(j + 1);
+      if (!ok) break;
+      const bool next = j + 1 < ntot;
+      for (int t = 0; t < nq && ok; ++t) {
+        // P_t(j), V(j) and, for S_t(j + 1), K(j + 1): one wait
+        ok = mbar_wait3(&bars.p_full[t], j & 1, &bars.v_full[j % kVS], (j / kVS) & 1,
+                        next ? &bars.k_full[(j + 1) % kKS] : nullptr, ((j + 1) / kKS) & 1, abort);
+        if (!ok) break;
+        fence_after();
+        issue_pv(t, j);
+        if (next) issue_s(t, j + 1);
+      }
+    }
+    if (!ok) {
+      // the issued MMAs complete before the TMEM is freed: they execute in
+      // issue order, and a tile's next P V waits for its softmax, which
+      // waits for its S, so each barrier has at most its last phase open
+      for (int t = 0; t < 2; ++t) {
+        if (s_issued[t] > 0) mbar_drain(&bars.s_full[t], (s_issued[t] - 1) & 1);
+        if (pv_issued[t] > 0) mbar_drain(&bars.pv_done[t], (pv_issued[t] - 1) & 1);
+      }
+    }
+  };
 
   if (warp == kWarpTree) {
     // ------------------------------------------------------------ tree bookkeeping
@@ -282,6 +368,9 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.tree_info);
     }
+  } else if (warp == kWarpMma) {
+    if (lane == 0) run_issuer();
+    __syncwarp();
   } else if (warp == kWarpK || warp == kWarpV) {
     // ------------------------------------------------------------ producers
     const bool isk = (warp == kWarpK);
@@ -354,92 +443,6 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
     if (lane == 0) {
       if (isk) mbar_drain(&bars.q_full, 0);
       for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j) mbar_drain(&full[j % NS], (j / NS) & 1);
-    }
-    __syncwarp();
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      bool ok = true;
-      int ntot = nprefix;
-      bool tree_known = !has_tree;
-      // the tree tiles follow the prefix tiles; their count is known once
-      // the tree warp has built U
-      auto know = [&](int upto) -> bool {
-        if (!tree_known && upto >= nprefix) {
-          if (!mbar_wait(&bars.tree_info, 0, abort)) return false;
-          ntot += (bars.nU + kKeys - 1) / kKeys;
-          tree_known = true;
-        }
-        return true;
-      };
-      const uint32_t idesc_qk = instr_desc(kRows, kKeys, 0, 0);
-      const uint32_t idesc_pv = instr_desc(kRows, kD, 0, 1);
-      int s_issued[2] = {0, 0}, pv_issued[2] = {0, 0};
-      // S_t(j) = Q_t K_j^T into S_t
-      auto issue_s = [&](int t, int j) {
-        const uint32_t sq = base + kSmemQ + t * kTileBytes;
-        const uint32_t sk = base + kSmemK + (j % kKS) * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_bf16(tmem + col_s(t), smem_desc(sq + off, 16, 1024), smem_desc(sk + off, 16, 1024), idesc_qk,
-                   kk > 0);
-        }
-        mma_commit(&bars.s_full[t]);
-        ++s_issued[t];
-      };
-      // O_t += P_t(j) V_j, P_t read from the first 64 columns of S_t
-      auto issue_pv = [&](int t, int j) {
-        const uint32_t sv = base + kSmemV + (j % kVS) * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, smem_desc(sv + kk * 2048, kHalfBytes, 1024),
-                      idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars.pv_done[t]);
-        ++pv_issued[t];
-      };
-      ok = know(0);
-      if (ok && ntot > 0) ok = mbar_wait(&bars.q_full, 0, abort);
-      if (ok && ntot > 0) {
-        ok = mbar_wait(&bars.k_full[0], 0, abort);
-        if (ok) {
-          fence_after();
-          for (int t = 0; t < nq; ++t) issue_s(t, 0);
-          mma_commit(&bars.k_empty[0]);
-        }
-      }
-      for (int j = 0; ok; ++j) {
-        ok = know(j);
-        if (!ok || j >= ntot) break;
-        ok = know(j + 1);
-        if (!ok) break;
-        const bool next = j + 1 < ntot;
-        ok = mbar_wait(&bars.v_full[j % kVS], (j / kVS) & 1, abort);
-        if (ok && next) ok = mbar_wait(&bars.k_full[(j + 1) % kKS], ((j + 1) / kKS) & 1, abort);
-        for (int t = 0; t < nq && ok; ++t) {
-          ok = mbar_wait(&bars.p_full[t], j & 1, abort);
-          if (!ok) break;
-          fence_after();
-          issue_pv(t, j);
-          if (t == nq - 1) mma_commit(&bars.v_empty[j % kVS]);
-          if (next) {
-            // S_t(j + 1) overwrites P_t(j)
-            ok = mbar_wait(&bars.pv_done[t], j & 1, abort);
-            if (!ok) break;
-            fence_after();
-            issue_s(t, j + 1);
-            if (t == nq - 1) mma_commit(&bars.k_empty[(j + 1) % kKS]);
-          }
-        }
-      }
-      if (!ok) {
-        // the issued MMAs complete before the TMEM is freed (each tile's last
-        // S and last P V are the only ones that can still be in flight)
-        for (int t = 0; t < 2; ++t) {
-          if (s_issued[t] > 0) mbar_drain(&bars.s_full[t], (s_issued[t] - 1) & 1);
-          if (pv_issued[t] > 0) mbar_drain(&bars.pv_done[t], (pv_issued[t] - 1) & 1);
-        }
-      }
     }
     __syncwarp();
   } else if (qt < nq) {
@@ -578,7 +581,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
       if (lane == 0) mbar_arrive(&bars.p_full[qt]);
     }
     // ------------------------------------------------------------ epilogue
-    // S_t(ntot - 1) was issued after P_t(ntot - 2) V completed, so phase
+    // S_t(ntot - 1) executed after P_t(ntot - 2) V (issue order), so phase
     // ntot - 1 of pv_done is the next one to complete
     if (ok && ntot > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done[qt], (ntot - 1) & 1, abort));
     fence_after();

@@ -35,7 +35,8 @@
 //              slot of its parent.
 // A K stage is released when its S = Q K^T completes, a V stage when its
 // P V completes, so the loads of later tiles start while earlier tiles are
-// in the softmax.  Online softmax in base 2 with a lazily updated maximum
+// in the softmax.  S(j+2) reuses the TMEM buffer that P(j) is read from; it
+// is issued right behind P(j) V (MMAs of one thread execute in issue order).  Online softmax in base 2 with a lazily updated maximum
 // per row half: O_h and its row sum are rescaled only when the half's
 // maximum grows by more than 2^8, which keeps P <= 256 (exact in the final
 // O / l).  P_h is written as bf16 over the first 32 columns of the half's
@@ -471,7 +472,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       for (int j = 0; ok; ++j) {
         ok = know(j);
         if (!ok || j >= ntot) break;
-        ok = mbar_wait(&bars.v_full[j % kVS], (j / kVS) & 1, abort);
+        // V(j) and the first half's P(j) in one wait
+        ok = mbar_wait3(&bars.v_full[j % kVS], (j / kVS) & 1, &bars.p_full[j & 1][0], (j >> 1) & 1, nullptr, 0u,
+                        abort);
         const uint32_t sv = base + kSmemV + (j % kVS) * kTileBytes;
         // O_h += P_h V_h: P_h (128 rows x 64 keys, bf16 pairs) sits in the
         // first 32 columns of the half's own S columns 64 h ..; V_h is rows
@@ -480,7 +483,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         // even when the second half never comes.
         bool any = false;
         for (int h = 0; h < 2 && ok; ++h) {
-          ok = mbar_wait(&bars.p_full[j & 1][h], (j >> 1) & 1, abort);
+          if (h > 0) ok = mbar_wait(&bars.p_full[j & 1][h], (j >> 1) & 1, abort);
           if (!ok) break;
           fence_after();
           const uint32_t od = tmem + (h ? kColO1 : kColO0);
@@ -502,10 +505,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         if (!ok) break;
         if (jn < ntot) {
           ok = mbar_wait(&bars.k_full[jn % kKS], (jn / kKS) & 1, abort);
-          // S(jn) overwrites the buffer P(j) is read from
-          if (ok) ok = mbar_wait(&bars.pv_done, j & 1, abort);
           if (!ok) break;
           fence_after();
+          // S(jn) overwrites the buffer P(j) is read from: MMAs of this
+          // thread execute in issue order, so it is queued right behind P(j) V
           issue_s(jn);
         }
       }

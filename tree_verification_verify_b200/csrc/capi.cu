@@ -69,8 +69,11 @@ tv_status check_attn(const tv_attn_args* a) {
 }
 
 // Time of one 128-key tile in a two-tile CTA (both row tiles), in units of
-// the same tile in a one-tile CTA.
-constexpr double kPairTile = 1.2;
+// the same tile in a one-tile CTA, and the two-tile CTA's fixed cost (start,
+// first loads, a two-round merge) in the same unit; measured on B200 with the
+// long-context and Llama-3-8B-shaped workloads.
+constexpr double kPairTile = 1.5;
+constexpr double kPairFixed = 6.0;
 
 AttnPlan plan_attn(const tv_attn_args* a) {
   AttnPlan pl;
@@ -122,7 +125,8 @@ AttnPlan plan_attn(const tv_attn_args* a) {
           if (act <= 0) continue;
           const int64_t u = form ? units_pair : units;
           const double waves = static_cast<double>((u + act - 1) / act);
-          const double cost = waves * (3.0 + static_cast<double>(lt) * (form ? kPairTile : 1.0));
+          const double cost = waves * (form ? kPairFixed + static_cast<double>(lt) * kPairTile
+                                            : 3.0 + static_cast<double>(lt));
           if (cost < best) { best = cost; best_len = lt; pl.pair = form == 1; }
         }
       }

@@ -168,6 +168,39 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, ui
       : "memory");
 }
 
+// mbarrier.test_wait (non-blocking) on phase `parity`.
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on up to three barriers at once (a null barrier counts as
+// complete).  The tests of one poll are independent instructions, so while
+// TMA writes stream into shared memory (which makes each barrier test slow)
+// the three checks cost about as much as one.  False when the CTA aborted or
+// the limit expired (then the abort flag is raised).
+__device__ __forceinline__ bool mbar_wait3(uint64_t* a, uint32_t pa, uint64_t* b, uint32_t pb, uint64_t* c,
+                                           uint32_t pc, volatile int* abort) {
+  bool da = a == nullptr, db = b == nullptr, dc = c == nullptr;
+  for (uint32_t it = 0; it < kWaitLimit; ++it) {
+    const bool ta = da || mbar_test(a, pa);
+    const bool tb = db || mbar_test(b, pb);
+    const bool tc_ = dc || mbar_test(c, pc);
+    da = ta; db = tb; dc = tc_;
+    if (da && db && dc) return true;
+    if ((it & 255u) == 255u && *abort) return false;
+  }
+  *abort = 1;
+  return false;
+}
+
 // Wait used while draining after an abort: bounded, ignores the abort flag.
 __device__ __forceinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
   const uint32_t a = smem_u32(b);
