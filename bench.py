@@ -553,6 +553,34 @@ def time_commit(step, K, W, flush):
     return tot / K, moved
 
 
+def expansion_ablation(step):
+    """The SpecExec page's ablation on the synthetic rows: the same 16 calls
+    of draft rows build one tree best-first and one by beam search; each
+    tree's sum of path probabilities is the expected number of accepted
+    tokens when the target distribution equals the draft's.  Also the beam
+    build's time (one build, CUDA events)."""
+    tv, ec = step.tv, step.ec
+    out = {}
+    for mode in ("bestfirst", "beam"):
+        st = tv.tree_expand_init(ec.budget, ec.V, ec.Bsel, device=step.dev)
+        def build():
+            tv.tree_expand_init(ec.budget, ec.V, ec.Bsel, state=st)
+            for k, z in enumerate(step.exp_logits):
+                rows = step.exp_root if k == 0 else st.frontier
+                tv.tree_expand_topb(st, z, rows, mode=mode)
+        build()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        build()
+        e1.record()
+        torch.cuda.synchronize()
+        n = int(st.n_nodes.item())
+        out[mode] = {"nodes": n, "expected_accepted": round(float(torch.exp(st.logp[1:n]).sum().item()), 4),
+                     "build_us": round(e0.elapsed_time(e1) * 1e3, 1)}
+    return out
+
+
 def call_summary(step, times, world):
     """Per-call mean times (max over ranks) with their work and roofline
     fractions."""
@@ -580,6 +608,7 @@ def call_summary(step, times, world):
             "us": round(ms["expand"] * 1e3, 2), "rounds": len(step.exp_logits),
             "gbs": round(step.expand_bytes / t / 1e9, 1), "algorithmic_bytes": step.expand_bytes,
             "nodes_per_s": n_new / t, **roofline_fracs(t, step.expand_bytes)}
+        out["tree_expand_topb"]["ablation_bestfirst_vs_beam"] = expansion_ablation(step)
     return ms, out
 
 

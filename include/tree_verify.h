@@ -267,9 +267,17 @@ TV_API tv_status tree_accept_noalloc(const tv_accept_args* a, tv_stream_t stream
  * is not yet in the tree or was expanded before is skipped
  * (TV_DEV_BAD_ROW); a row with a non-finite logit is skipped
  * (TV_DEV_NONFINITE).
+ * mode TV_EXPAND_BEAM (the SpecExec page's ablation, "Replace parallel SSSP
+ * tree search with standard beam search") instead ranks only the children of
+ * this call's rows: the sel best of them are appended, in the same order,
+ * and no candidate is carried to later calls (the rows of one call are one
+ * depth of the beam).  Mixing the modes between calls of one tree is not
+ * supported.
  * Limits: 1 <= budget <= 8192, 1 <= V <= 262144, 1 <= Bsel,
  * draft_temperature > 0.
  * ---------------------------------------------------------------------- */
+typedef enum { TV_EXPAND_BESTFIRST = 0, TV_EXPAND_BEAM = 1 } tv_expand_mode;
+
 typedef struct {
   int32_t V, R, Bsel, budget;
   float draft_temperature;
@@ -283,6 +291,7 @@ typedef struct {
   int32_t* frontier;
   int32_t* n_appended;
   uint32_t* dev_status;
+  int32_t mode;               /* tv_expand_mode */
 } tv_expand_args;
 
 TV_API size_t tree_expand_pool_bytes(int32_t budget, int32_t V);

@@ -30,6 +30,11 @@ Reading of "top-B": Bsel nodes are appended per round (batched Dijkstra with
 a carried pool), not the top-B children of the current depth (beam search).
 The budget counts the root.
 
+Beam mode (the page's ablation "Replace parallel SSSP tree search with
+standard beam search"): a call ranks only the children of its own rows (the
+current depth's beam) by the same scores and order, appends the best
+min(Bsel, budget - n_nodes) of them, and carries nothing to later calls.
+
 Status bits: BAD_ROW (8) for a row whose node is not in the tree or was
 already expanded (the row is skipped); NONFINITE (4) for a row holding a
 non-finite logit (skipped; the node still counts as expanded).
@@ -69,15 +74,22 @@ def row_scores(logp_n: float, z, tau: float):
     return (logp_n + x) - lse
 
 
-def expand_call(st: ExpandState, draft_logits, row_node, Bsel: int, tau: float = 1.0):
-    """One round.  draft_logits [R][V], row_node [R] (-1 = no row).
+def expand_call(st: ExpandState, draft_logits, row_node, Bsel: int, tau: float = 1.0,
+                mode: str = "bestfirst"):
+    """One round.  draft_logits [R][V], row_node [R] (-1 = no row); mode
+    "bestfirst" (carried pool) or "beam" (this call's rows only).
     Returns the appended node indices (the next frontier)."""
+    if mode not in ("bestfirst", "beam"):
+        raise ValueError(mode)
     Zd = draft_logits
     rows = [int(x) for x in _i64(row_node)]
     rem = st.budget - st.n_nodes
-    sc = [st.pool_score]
-    pa = [st.pool_parent]
-    tk = [st.pool_token]
+    if mode == "beam":
+        sc, pa, tk = [np.zeros(0)], [np.zeros(0, dtype=np.int64)], [np.zeros(0, dtype=np.int64)]
+    else:
+        sc = [st.pool_score]
+        pa = [st.pool_parent]
+        tk = [st.pool_token]
     for r, n in enumerate(rows):
         if n < 0:
             continue
@@ -110,7 +122,7 @@ def expand_call(st: ExpandState, draft_logits, row_node, Bsel: int, tau: float =
         st.token.append(int(tok[r]))
         st.logp.append(float(score[r]))
         new.append(st.n_nodes - 1)
-    keep = st.budget - st.n_nodes
+    keep = st.budget - st.n_nodes if mode == "bestfirst" else 0
     st.pool_score = score[sel:sel + keep]
     st.pool_parent = par[sel:sel + keep]
     st.pool_token = tok[sel:sel + keep]

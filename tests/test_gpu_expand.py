@@ -32,7 +32,7 @@ def _lib():
     build.build()
 
 
-def _compare_build(V, Bsel, budget, logits_fn, tau=1.0, root_token=0):
+def _compare_build(V, Bsel, budget, logits_fn, tau=1.0, root_token=0, mode="bestfirst"):
     """Run GPU and oracle round by round on identical rows.  logits_fn(call,
     R) returns [R][V] fp32 rows for the frontier of that call (identical
     frontiers on both sides, checked every round)."""
@@ -47,8 +47,8 @@ def _compare_build(V, Bsel, budget, logits_fn, tau=1.0, root_token=0):
     while os_.n_nodes < budget and frontier:
         z = logits_fn(call, len(frontier))
         rows = torch.tensor(frontier, dtype=torch.int32, device="cuda")
-        tv.tree_expand_topb(st, z.cuda(), rows, draft_temperature=tau, dev_status=status)
-        new = expand_call(os_, z, frontier, Bsel, tau)
+        tv.tree_expand_topb(st, z.cuda(), rows, draft_temperature=tau, dev_status=status, mode=mode)
+        new = expand_call(os_, z, frontier, Bsel, tau, mode=mode)
         torch.cuda.synchronize()
         gap = os_.gaps[-1]
         nap = int(st.n_appended.item())
@@ -207,3 +207,45 @@ def test_signed_zero_logits_tie_by_token():
     # the first round takes token 40's... no: the root row's three best are
     # the zeros at tokens 3, 10 and 20 (0 > -4 and token order inside the tie)
     assert os_.token[1:4] == [3, 10, 20]
+
+
+@pytest.mark.parametrize("V,Bsel,budget,sigma", [
+    (256, 8, 64, 3.0),          # the tiny workload's shape
+    (37, 5, 101, 2.0),          # ragged vocabulary
+    (5000, 200, 1200, 4.0),     # Bsel above one merge sub-step
+    (32000, 128, 2048, 4.0),    # the SpecExec-shaped build
+])
+def test_beam_mode(V, Bsel, budget, sigma):
+    """Beam mode (the SpecExec page's ablation: standard beam search) against
+    the oracle's beam mode, every round: only the call's own rows are
+    ranked, nothing is carried."""
+    ec = expand_case(V, Bsel, budget, sigma, seed=V + 1)
+    compared, near, st, os_ = _compare_build(V, Bsel, budget, lambda c, R: ec.round_logits(c, R), mode="beam")
+    print(f"beam V={V} Bsel={Bsel} budget={budget}: {compared} rounds compared, near-tie stop: {near}")
+    assert not near and compared >= 1 and os_.n_nodes == budget
+
+
+def test_beam_mode_keeps_less_mass_than_best_first():
+    """On the same rows per call, the best-first tree's total path
+    probability (the expected accepted length when the target matches the
+    draft) exceeds the beam tree's: the page's ablation, qualitatively."""
+    import tree_verification_verify_b200 as tv
+    V, Bsel, budget = 32000, 128, 2048
+    ec = expand_case(V, Bsel, budget, 4.0, seed=5)
+    mass = {}
+    for mode in ("bestfirst", "beam"):
+        st = tv.tree_expand_init(budget, V, Bsel)
+        frontier = torch.zeros(1, dtype=torch.int32, device="cuda")
+        for call in range(ec.n_calls()):
+            z = ec.round_logits(call, frontier.numel()).cuda()
+            f, k = tv.tree_expand_topb(st, z, frontier, mode=mode)
+            kk = int(k.item())
+            if kk == 0:
+                break
+            frontier = f[:kk].clone()
+        torch.cuda.synchronize()
+        n = int(st.n_nodes.item())
+        mass[mode] = float(torch.exp(st.logp[1:n]).sum().item())
+    print(f"expected accepted length (sum of path probabilities): best-first {mass['bestfirst']:.3f}, "
+          f"beam {mass['beam']:.3f}")
+    assert mass["bestfirst"] > mass["beam"]

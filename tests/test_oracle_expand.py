@@ -257,3 +257,65 @@ def test_nonfinite_row_consumes_its_node():
     parents = [st.parent[i] for i in new]
     assert 1 not in parents and 2 in parents
     assert 1 in st.expanded and 2 in st.expanded
+
+
+def _path_rows(V, seed):
+    """Draft logits keyed by the node's token path (order-independent)."""
+    def rows(path):
+        h = (seed * 1_000_003 + hash(path)) % (2 ** 32)
+        return np.random.default_rng(h).normal(0.0, 2.0, V)
+    return rows
+
+
+@pytest.mark.parametrize("V,Bsel,budget,seed", [(4, 3, 30, 0), (7, 5, 60, 1), (3, 9, 40, 2), (16, 6, 50, 3)])
+def test_beam_mode_matches_beam_search(V, Bsel, budget, seed):
+    """Beam mode, round by round with the frontier as the rows, builds the
+    tree that an independent path-level beam search builds (each depth keeps
+    the best Bsel children of the previous depth)."""
+    rows = _path_rows(V, seed)
+    st = ExpandState(budget)
+    frontier = [0]
+    while st.n_nodes < budget and frontier:
+        paths = _paths(st)
+        frontier = expand_call(st, np.stack([rows(paths[n]) for n in frontier]), frontier, Bsel, mode="beam")
+        assert len(st.pool_score) == 0
+    bpaths, blogp = _beam(V, Bsel, budget, rows)
+    got = _paths(st)
+    assert got == bpaths
+    np.testing.assert_allclose(st.logp, blogp, rtol=0, atol=1e-12)
+
+
+def test_beam_mode_with_one_beam_is_greedy_decoding():
+    """Bsel = 1: every call appends the single best child of the one
+    frontier node, so the tree is the chain of row argmaxes."""
+    V, budget = 9, 12
+    rows = _path_rows(V, 7)
+    st = ExpandState(budget)
+    frontier = [0]
+    while st.n_nodes < budget and frontier:
+        paths = _paths(st)
+        frontier = expand_call(st, np.stack([rows(paths[n]) for n in frontier]), frontier, 1, mode="beam")
+    path = ()
+    for i in range(1, budget):
+        assert st.parent[i] == i - 1
+        assert st.token[i] == int(np.argmax(rows(path)))
+        path = path + (st.token[i],)
+
+
+def test_beam_mode_never_revisits_an_earlier_depth():
+    """With the root's runners-up far better than every grandchild, best
+    first takes them in the second round while beam mode does not."""
+    V, Bsel, budget = 6, 2, 6
+
+    def rows(path):
+        z = np.full(V, -8.0)
+        if path == ():
+            z[:4] = [3.0, 2.9, 2.8, 2.7]
+        return z
+    for mode, want_root_children in (("bestfirst", 4), ("beam", 2)):
+        st = ExpandState(budget)
+        frontier = [0]
+        while st.n_nodes < budget and frontier:
+            paths = _paths(st)
+            frontier = expand_call(st, np.stack([rows(paths[n]) for n in frontier]), frontier, Bsel, mode=mode)
+        assert sum(1 for q in st.parent[1:] if q == 0) == want_root_children

@@ -21,7 +21,7 @@ from typing import Optional
 import torch
 
 __all__ = ["lib", "version", "status_string", "tree_verify_attn", "tree_accept", "tree_accept_noalloc",
-           "tree_expand_init", "tree_expand_topb", "ExpandState", "tree_commit_kv", "philox_uniforms",
+           "tree_expand_init", "tree_expand_topb", "ExpandState", "EXPAND_MODES", "tree_commit_kv", "philox_uniforms",
            "TVError", "MODES"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -68,7 +68,10 @@ class ExpandArgs(ctypes.Structure):
                 ("row_node", c_vp),
                 ("n_nodes", c_vp), ("parent", c_vp), ("token", c_vp), ("logp", c_vp),
                 ("pool", c_vp), ("pool_bytes", c_size),
-                ("frontier", c_vp), ("n_appended", c_vp), ("dev_status", c_vp)]
+                ("frontier", c_vp), ("n_appended", c_vp), ("dev_status", c_vp), ("mode", c_i32)]
+
+
+EXPAND_MODES = {"bestfirst": 0, "beam": 1}
 
 
 class CommitArgs(ctypes.Structure):
@@ -396,14 +399,16 @@ class ExpandState:
     def pool_ptr(self) -> int:
         return _aligned_ptr(self._pool)
 
-    def args(self, draft_logits=None, row_node=None, temperature: float = 1.0, dev_status=None):
+    def args(self, draft_logits=None, row_node=None, temperature: float = 1.0, dev_status=None,
+             mode: str = "bestfirst"):
         R = 0 if row_node is None else int(row_node.numel())
         ld = draft_logits.stride(0) if draft_logits is not None else self.V
         return ExpandArgs(self.V, R, self.Bsel, self.budget, float(temperature),
                           _ptr(draft_logits), ld, _ptr(row_node),
                           self.n_nodes.data_ptr(), self.parent.data_ptr(), self.token.data_ptr(),
                           self.logp.data_ptr(), self.pool_ptr, self.pool_bytes,
-                          self.frontier.data_ptr(), self.n_appended.data_ptr(), _ptr(dev_status))
+                          self.frontier.data_ptr(), self.n_appended.data_ptr(), _ptr(dev_status),
+                          EXPAND_MODES[mode])
 
 
 def tree_expand_init(budget: int, V: int, Bsel: int, root_token: int = 0, device=None,
@@ -419,15 +424,19 @@ def tree_expand_init(budget: int, V: int, Bsel: int, root_token: int = 0, device
 
 
 def tree_expand_topb(state: ExpandState, draft_logits, row_node, draft_temperature: float = 1.0,
-                     dev_status=None, stream=None):
+                     dev_status=None, stream=None, mode: str = "bestfirst"):
     """One round (include/tree_verify.h, tree_expand_topb).  draft_logits fp32
-    [R][V] with contiguous rows, row_node int32 [R].  Returns the state's
-    frontier and n_appended tensors (device)."""
+    [R][V] with contiguous rows, row_node int32 [R]; mode "bestfirst"
+    (batched best-first with a carried pool) or "beam" (the children of this
+    round's rows only).  Returns the state's frontier and n_appended tensors
+    (device)."""
     _need_cuda(draft_logits, row_node)
     if draft_logits.dtype != torch.float32 or draft_logits.stride(-1) != 1:
         raise TVError("draft_logits must be fp32 with contiguous rows")
+    if mode not in EXPAND_MODES:
+        raise TVError(f"mode must be one of {sorted(EXPAND_MODES)}")
     row_node = _i32(row_node)
-    a = state.args(draft_logits, row_node, draft_temperature, dev_status)
+    a = state.args(draft_logits, row_node, draft_temperature, dev_status, mode)
     _check(lib().tree_expand_topb(ctypes.byref(a), None, 0, _stream(stream)), "tree_expand_topb")
     return state.frontier, state.n_appended
 

@@ -295,6 +295,7 @@ tv_status check_expand(const tv_expand_args* a, bool need_rows) {
   if (a->V < 1 || a->budget < 1 || a->Bsel < 1 || a->R < 0) return TV_ERR_INVALID_ARG;
   if (a->V > 262144 || a->budget > 8192) return TV_ERR_UNSUPPORTED;
   if (!(a->draft_temperature > 0.f) || !std::isfinite(a->draft_temperature)) return TV_ERR_INVALID_ARG;
+  if (a->mode != TV_EXPAND_BESTFIRST && a->mode != TV_EXPAND_BEAM) return TV_ERR_INVALID_ARG;
   if (!a->n_nodes || !a->parent || !a->token || !a->logp || !a->pool) return TV_ERR_INVALID_ARG;
   if (a->pool_bytes < tv::expand_pool_bytes(a->budget, a->V)) return TV_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(a->pool) & 255u) != 0) return TV_ERR_WORKSPACE;

@@ -19,6 +19,10 @@
 //                        bitonic sort of the K into the node's list (a
 //                        boundary bin too crowded for shared memory falls
 //                        back to a radix select on the 32-bit key);
+// Beam mode (the SpecExec page's ablation: standard beam search) ranks only
+// the children of the call's own rows: each row's list holds its best
+// min(V, Bsel) tokens and the merge reads the lists stamped by this call.
+//
 //   expand_merge_kernel  one CTA: repeatedly take the best s <= 128
 //                        candidates of the union.  The s-th best list head
 //                        bounds the s-th best candidate, so only the <= s
@@ -35,9 +39,16 @@ struct NodeMeta {
   int32_t len;        // entries in the node's sorted list (0: not expanded)
   int32_t cursor;     // first entry not yet taken
   int32_t expanded;   // set once a row for the node has been consumed
-  int32_t pad;
+  int32_t stamp;      // number of the call whose row built the list
   double lse;         // logsumexp of the node's row / tau
 };
+
+// Pool header: calls made since tree_expand_init (stamps the lists, so
+// that beam mode takes only the lists its own rows built).
+struct PoolHeader {
+  int32_t calls;
+};
+constexpr size_t kPoolHeaderBytes = 256;
 
 struct ListEntry {
   float z;
@@ -58,12 +69,13 @@ __host__ __device__ inline int64_t expand_kcap(int budget, int V) {
   return k < 1 ? 1 : k;
 }
 __host__ __device__ inline size_t expand_lists_offset(int budget) {
-  const size_t m = static_cast<size_t>(budget) * sizeof(NodeMeta);
+  const size_t m = kPoolHeaderBytes + static_cast<size_t>(budget) * sizeof(NodeMeta);
   return (m + 255) & ~static_cast<size_t>(255);
 }
 
 struct ExpandParams {
   int V, R, Bsel, budget;
+  int beam;               // TV_EXPAND_BEAM: rank this call's rows only
   float tau;
   const float* logits; int64_t ld;
   const int32_t* row_node;
@@ -71,6 +83,7 @@ struct ExpandParams {
   int32_t* parent;
   int32_t* token;
   double* logp;
+  PoolHeader* header;
   NodeMeta* meta;
   ListEntry* lists;
   int64_t kcap;
@@ -294,7 +307,9 @@ expand_rows_kernel(ExpandParams p) {
     return;
   }
   const int V = p.V;
-  const int K = min(V, p.budget - n0);
+  // best-first: every candidate that can still be taken; beam: this call
+  // takes at most Bsel, and its lists are not used later
+  const int K = p.beam ? min(min(V, p.Bsel), p.budget - n0) : min(V, p.budget - n0);
   if (K <= 0) return;
   const float* row = p.logits + static_cast<int64_t>(r) * p.ld;
   const bool vec = (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
@@ -472,6 +487,7 @@ expand_rows_kernel(ExpandParams p) {
     p.meta[node].len = K;
     p.meta[node].cursor = 0;
     p.meta[node].lse = lse;
+    p.meta[node].stamp = __ldcg(&p.header->calls) + 1;
   }
 }
 
@@ -560,13 +576,25 @@ expand_merge_kernel(ExpandParams p) {
   const int n0 = *p.n_nodes;
   const int rem = p.budget - n0;
   const int total = rem > 0 ? min(p.Bsel, rem) : 0;
+  const int stamp = __ldcg(&p.header->calls) + 1;    // this call's number
   int appended = 0;
   while (appended < total) {
     const int s = min(kMergeStep, total - appended);
     // 1. list heads of every expanded node with entries left
     if (tid == 0) { sh.cnt[0] = 0; sh.cnt[1] = 0; sh.cnt[2] = 0; }
     __syncthreads();
-    for (int nd = tid; nd < n0; nd += blockDim.x) {
+    // best-first: every expanded node's list; beam: only the lists built by
+    // this call's rows (each node once)
+    const int nh = p.beam ? p.R : n0;
+    for (int h = tid; h < nh; h += blockDim.x) {
+      int nd = h;
+      if (p.beam) {
+        nd = p.row_node[h];
+        if (nd < 0 || nd >= n0 || __ldcg(&p.meta[nd].stamp) != stamp) continue;
+        bool dup = false;
+        for (int h2 = 0; h2 < h && !dup; ++h2) dup = (p.row_node[h2] == nd);
+        if (dup) continue;
+      }
       const int len = __ldcg(&p.meta[nd].len);
       const int cur = __ldcg(&p.meta[nd].cursor);
       if (cur < len) {
@@ -679,9 +707,11 @@ expand_merge_kernel(ExpandParams p) {
     if (S < s) break;
   }
   for (int i = appended + tid; i < p.Bsel; i += blockDim.x) p.frontier[i] = -1;
+  __syncthreads();
   if (tid == 0) {
     *p.n_nodes = n0 + appended;
     *p.n_appended = appended;
+    p.header->calls = stamp;
   }
 }
 
@@ -689,10 +719,11 @@ __global__ void expand_init_kernel(ExpandParams p, int root_token) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < p.budget) {
     NodeMeta m;
-    m.len = 0; m.cursor = 0; m.expanded = 0; m.pad = 0; m.lse = 0.0;
+    m.len = 0; m.cursor = 0; m.expanded = 0; m.stamp = 0; m.lse = 0.0;
     p.meta[i] = m;
   }
   if (i == 0) {
+    p.header->calls = 0;
     *p.n_nodes = 1;
     p.parent[0] = -1;
     p.token[0] = root_token;
@@ -710,11 +741,13 @@ size_t expand_pool_bytes(int budget, int V) {
 static ExpandParams make_params(const tv_expand_args* a) {
   ExpandParams p;
   p.V = a->V; p.R = a->R; p.Bsel = a->Bsel; p.budget = a->budget;
+  p.beam = a->mode == TV_EXPAND_BEAM;
   p.tau = a->draft_temperature;
   p.logits = a->draft_logits; p.ld = a->ld_logits;
   p.row_node = a->row_node;
   p.n_nodes = a->n_nodes; p.parent = a->parent; p.token = a->token; p.logp = a->logp;
-  p.meta = static_cast<NodeMeta*>(a->pool);
+  p.header = static_cast<PoolHeader*>(a->pool);
+  p.meta = reinterpret_cast<NodeMeta*>(static_cast<unsigned char*>(a->pool) + kPoolHeaderBytes);
   p.lists = reinterpret_cast<ListEntry*>(static_cast<unsigned char*>(a->pool) + expand_lists_offset(a->budget));
   p.kcap = expand_kcap(a->budget, a->V);
   p.frontier = a->frontier; p.n_appended = a->n_appended;
