@@ -19,7 +19,11 @@ the 8 TB/s / 2.25 PFLOP/s denominators.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--config longctx|longctx_sparse|specexec70b|serving|llama3_8b|tiny]
-                    [--only] [--no-cpu-baseline]
+                    [--only] [--no-cpu-baseline] [--split-prefix]
+
+--split-prefix times the long-context attention with each sequence's prefix
+split across the N ranks (prefix-only partials, NCCL all-gather, the
+log-sum-exp merge kernel): strong scaling of one layer's verification.
 
 Timing: the step's calls are captured once into one CUDA graph (and each
 call into a graph of its own); W untimed warm-up steps, then K steps of the
@@ -952,6 +956,73 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_split_prefix(args, rank, world, dev, flush):
+    """Strong scaling of the long-context attention: rank r attends to its
+    slice [r * Lmax / N, (r + 1) * Lmax / N) of every sequence's prefix
+    (prefix-only partials; the last rank also takes the tree keys), the
+    partials are all-gathered over NCCL and merged by log-sum-exp with
+    tree_verify_attn_merge.  A step = partial + all-gather + merge, timed
+    with CUDA events (max over ranks); `value` counts each tree token once."""
+    import tree_verification_verify_b200 as tv
+    from synth import config_attn_case
+    a = config_attn_case("longctx", seed=0, device=dev)
+    B, T, Hq, d = a.q.shape
+    Lmax = a.k_cache.shape[1]
+    lo, hi = (rank * Lmax) // world, ((rank + 1) * Lmax) // world
+    L = a.prefix_len.cpu().numpy()
+    pl = torch.from_numpy(np.clip(L - lo, 0, hi - lo).astype(np.int32)).to(dev)
+    kc, vc = a.k_cache[:, lo:hi], a.v_cache[:, lo:hi]
+    part_o = torch.empty_like(a.q)
+    part_l = torch.empty(B, T, Hq, dtype=torch.float32, device=dev)
+    all_o = torch.empty((world,) + tuple(a.q.shape), dtype=a.q.dtype, device=dev)
+    all_l = torch.empty(world, B, T, Hq, dtype=torch.float32, device=dev)
+    out = torch.empty_like(a.q)
+    lse = torch.empty_like(part_l)
+
+    def one():
+        tv.tree_verify_attn(a.q, kc, vc, pl, a.k_tree, a.v_tree, a.parent, out=part_o, lse=part_l,
+                            prefix_only=(rank != world - 1))
+        if world > 1:
+            import torch.distributed as dist
+            dist.all_gather_into_tensor(all_o, part_o)
+            dist.all_gather_into_tensor(all_l, part_l)
+        else:
+            all_o[0].copy_(part_o)
+            all_l[0].copy_(part_l)
+        tv.tree_verify_attn_merge(all_o, all_l, out=out, lse=lse)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    ts = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        one()
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = max_over_ranks(statistics.fmean(ts), world)
+    flops, nbytes = attn_work(a.parent.cpu().numpy(), [int(x) for x in L], T, Hq, a.k_cache.shape[2], d,
+                              a.q.element_size())
+    line = {"metric": METRIC, "value": B * T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "longctx attention, prefix split across ranks: B=4 Hq=32 Hkv=8 d=128 bf16 "
+                                   "prefix=131072 T=256", "parallelism": f"prefix split x{world}",
+                       "l2": "256 MiB flush before every timed step (not timed)",
+                       "launch": "eager calls; NCCL all-gather of the partials"},
+            "roofline": {"bound": "tensor", "achieved": round(flops / (ms * 1e-3) / 1e12, 2),
+                         "peak": peaks()[1] * world, "unit": "TFLOP/s",
+                         "frac": round(flops / (ms * 1e-3) / 1e12 / (peaks()[1] * world), 4)},
+            "gpu_launches": (3 if world > 1 else 2) * args.steps}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main_roofline(step, ms, hbm, bf16, src):
     """The roofline object of the step's dominant call."""
     attn_s, acc_s = ms["attn"] * 1e-3, ms["accept"] * 1e-3
@@ -1019,6 +1090,8 @@ def main():
     ap.add_argument("--config", default="longctx", choices=CONFIG_NAMES)
     ap.add_argument("--only", action="store_true", help="time the main workload alone (no other configs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split-prefix", action="store_true",
+                    help="long-context attention with the prefix split across the ranks (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -1032,6 +1105,12 @@ def main():
     build.build()
     dev = torch.device("cuda", torch.cuda.current_device())
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    if args.split_prefix:
+        run_split_prefix(args, rank, world, dev, flush)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     clk = ClockSampler(local)
     clk.start()
     main_res = run_config(args.config, args, world, rank, dev, flush, args.steps, args.warmup, True)

@@ -132,6 +132,14 @@ typedef enum { TV_FP32 = 0, TV_BF16 = 1 } tv_dtype;
  * malformed gets NaN rows (TV_DEV_BAD_PARENT); a sequence whose prefix_len
  * is outside [0, Lmax] gets NaN rows and one whose n_nodes is outside
  * [0, T] gets none (TV_DEV_BAD_LEN).
+ *
+ * prefix_only = 1 computes a partial instead: each node attends to the
+ * prefix keys alone (no tree keys; parent[] is not read), for splitting a
+ * long prefix across GPUs (each rank passes its slice of the cache, e.g. a
+ * view from row lo, with prefix_len = the slice's length per sequence; one
+ * rank keeps prefix_only = 0 so the tree keys are counted once), then
+ * tree_verify_attn_merge.  A row with no keys (an empty slice) gets O = 0
+ * and lse = -inf.  Not with sparse_topk (TV_ERR_UNSUPPORTED).
  * ---------------------------------------------------------------------- */
 typedef struct {
   int32_t dtype;
@@ -152,11 +160,39 @@ typedef struct {
   float* lse;
   int32_t* sel_blocks;
   uint32_t* dev_status;
+  int32_t prefix_only;
 } tv_attn_args;
 
 TV_API size_t tree_verify_attn_workspace_size(const tv_attn_args* a);
 TV_API tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws_bytes,
                            tv_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * tree_verify_attn_merge
+ *
+ * Combines N attention partials over disjoint key sets of the same rows
+ * (the outputs and natural-log lse of tree_verify_attn calls on slices of a
+ * split prefix, gathered from the ranks) by their log-sum-exp:
+ *     M = max_r lse_r,  w_r = exp(lse_r - M),
+ *     out = sum_r w_r o_r / sum_r w_r,  lse = M + log sum_r w_r
+ * (the same algebra that merges a split prefix inside one GPU).  Layouts,
+ * all contiguous device memory: o_parts [N][B][T][Hq][d] (dtype),
+ * lse_parts [N][B][T][Hq] fp32, out [B][T][Hq][d] (dtype), lse [B][T][Hq]
+ * fp32 or NULL.  A row whose partials are all -inf gets out = 0 and
+ * lse = -inf; a NaN lse in any partial makes the row NaN.
+ * 1 <= N <= 64, d in {32, 64, 128}; other values TV_ERR_INVALID_ARG /
+ * TV_ERR_UNSUPPORTED.  No workspace; enqueues on `stream`.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int32_t dtype;
+  int32_t N, B, T, Hq, d;
+  const void* o_parts;
+  const float* lse_parts;
+  void* out;
+  float* lse;
+} tv_attn_merge_args;
+
+TV_API tv_status tree_verify_attn_merge(const tv_attn_merge_args* a, tv_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * tree_accept

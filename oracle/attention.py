@@ -32,6 +32,15 @@ kept for all heads of the group; with at most k blocks all are kept.  The
 node then attends to the kept blocks' keys plus its tree path, exactly as
 above.
 
+Prefix-only partial (for splitting a long prefix across GPUs, the long
+contexts the sparse verification page is about): with prefix_only the node
+attends to the prefix keys alone, K(i) = {0 .. L_b - 1}
+(parent[] is not read); a row with no keys has out = 0 and lse = -inf.
+Partials over disjoint key sets of the same rows combine by their
+log-sum-exp (merge_partials): with M = max_r lse_r and w_r = exp(lse_r - M),
+out = sum_r w_r out_r / sum_r w_r and lse = M + log sum_r w_r, which is the
+softmax over the union of the key sets.
+
 Malformed input (reported as bits of a status word, outputs defined):
   BAD_PARENT (1): parent[0] != -1, or a node whose parent chain does not
       reach the root through parent[j] in [0, j): its outputs are NaN.
@@ -122,7 +131,7 @@ def select_blocks(qi_group, kbar_bg, nblk, topk):
 
 def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent,
                      n_nodes=None, scale=0.0, sparse_topk=0, block_size=64,
-                     k_block_mean=None, rows=None, forced_sel=None):
+                     k_block_mean=None, rows=None, forced_sel=None, prefix_only=False):
     """Oracle for tree_verify_attn.
 
     Shapes: q [B][T][Hq][d], k_cache/v_cache [B][Lmax][Hkv][d],
@@ -176,17 +185,18 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent,
         bad_len = Lb < 0 or Lb > Lmax
         if bad_len:
             status |= ST_BAD_LEN
-        if n > 0 and P[b, 0] != -1:
-            status |= ST_BAD_PARENT
-        for i in range(1, n):
-            if P[b, i] < 0 or P[b, i] >= i:
+        if not prefix_only:
+            if n > 0 and P[b, 0] != -1:
                 status |= ST_BAD_PARENT
+            for i in range(1, n):
+                if P[b, i] < 0 or P[b, i] >= i:
+                    status |= ST_BAD_PARENT
         nblk = (Lb + block_size - 1) // block_size if not bad_len else 0
         for i in range(n):
             if rows is not None and (b, i) not in rows:
                 continue
             written[b, i] = True
-            path = ancestor_path(P[b], i)
+            path = [] if prefix_only else ancestor_path(P[b], i)
             if path is None or bad_len:
                 if path is None:
                     status |= ST_BAD_PARENT
@@ -207,6 +217,10 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent,
                     vp = Vc[b, :Lb, g]
                 keys = np.concatenate([kp, KT[b, path, g]], axis=0)
                 vals = np.concatenate([vp, VT[b, path, g]], axis=0)
+                if len(keys) == 0:
+                    out[b, i, g * G:(g + 1) * G] = 0.0
+                    lse[b, i, g * G:(g + 1) * G] = -np.inf
+                    continue
                 # the G query heads of group g, one row each: [G][|K(i)|]
                 s = (Q[b, i, g * G:(g + 1) * G] @ keys.T) * sc
                 m = np.max(s, axis=1, keepdims=True)
@@ -217,3 +231,23 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent,
     return dict(out=out, lse=lse, written=written, valid=valid,
                 sel=(sel if topk > 0 else None), sel_gap=(sel_gap if topk > 0 else None),
                 status=status)
+
+
+def merge_partials(outs, lses):
+    """Log-sum-exp merge of attention partials over disjoint key sets of the
+    same rows: outs [N][...][d], lses [N][...] (natural log).  Rows whose
+    partials all have lse = -inf get out = 0 and lse = -inf; a NaN lse
+    makes the row NaN."""
+    O = np.asarray(outs, dtype=np.float64)
+    Lz = np.asarray(lses, dtype=np.float64)
+    bad = np.any(np.isnan(Lz), axis=0)
+    M = np.max(np.where(np.isnan(Lz), -np.inf, Lz), axis=0)
+    Ms = np.where(np.isfinite(M), M, 0.0)
+    w = np.where(np.isfinite(Lz), np.exp(np.where(np.isfinite(Lz), Lz, 0.0) - Ms[None]), 0.0)
+    den = np.sum(w, axis=0)
+    num = np.sum(w[..., None] * np.nan_to_num(O), axis=0)
+    out = np.where(den[..., None] > 0, num / np.where(den > 0, den, 1.0)[..., None], 0.0)
+    lse = np.where(den > 0, Ms + np.log(np.where(den > 0, den, 1.0)), -np.inf)
+    out[bad] = np.nan
+    lse[bad] = np.nan
+    return out, lse

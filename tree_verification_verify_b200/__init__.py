@@ -20,7 +20,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["lib", "version", "status_string", "tree_verify_attn", "tree_accept", "tree_accept_noalloc",
+__all__ = ["lib", "version", "status_string", "tree_verify_attn", "tree_verify_attn_merge", "tree_accept", "tree_accept_noalloc",
            "tree_expand_init", "tree_expand_topb", "ExpandState", "EXPAND_MODES", "tree_commit_kv", "philox_uniforms",
            "TVError", "MODES"]
 
@@ -46,7 +46,12 @@ class AttnArgs(ctypes.Structure):
                 ("scale", c_f32), ("sparse_topk", c_i32), ("block_size", c_i32),
                 ("k_block_mean", c_vp),
                 ("out", c_vp), ("o_sb", c_i64), ("o_st", c_i64), ("o_sh", c_i64),
-                ("lse", c_vp), ("sel_blocks", c_vp), ("dev_status", c_vp)]
+                ("lse", c_vp), ("sel_blocks", c_vp), ("dev_status", c_vp), ("prefix_only", c_i32)]
+
+
+class AttnMergeArgs(ctypes.Structure):
+    _fields_ = [("dtype", c_i32), ("N", c_i32), ("B", c_i32), ("T", c_i32), ("Hq", c_i32), ("d", c_i32),
+                ("o_parts", c_vp), ("lse_parts", c_vp), ("out", c_vp), ("lse", c_vp)]
 
 
 class AcceptArgs(ctypes.Structure):
@@ -99,6 +104,7 @@ def lib() -> ctypes.CDLL:
                           "`python -m tree_verification_verify_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
         for name, args in (("tree_verify_attn", [ctypes.POINTER(AttnArgs), c_vp, c_size, c_vp]),
+                           ("tree_verify_attn_merge", [ctypes.POINTER(AttnMergeArgs), c_vp]),
                            ("tree_accept", [ctypes.POINTER(AcceptArgs), c_vp, c_size, c_vp]),
                            ("tree_accept_noalloc", [ctypes.POINTER(AcceptArgs), c_vp]),
                            ("tree_expand_topb", [ctypes.POINTER(ExpandArgs), c_vp, c_size, c_vp]),
@@ -196,11 +202,14 @@ def _aligned_ptr(buf: torch.Tensor) -> int:
 def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent, n_nodes=None,
                      scale: float = 0.0, sparse_topk: int = 0, block_size: int = 64,
                      k_block_mean=None, out=None, lse=None, want_lse: bool = True,
-                     sel_blocks=None, want_sel: bool = False, dev_status=None, stream=None):
+                     sel_blocks=None, want_sel: bool = False, dev_status=None, stream=None,
+                     prefix_only: bool = False):
     """Tree-masked attention (include/tree_verify.h, tree_verify_attn).
     Shapes: q [B][T][Hq][d], caches [B][Lmax][Hkv][d], tree K/V [B][T][Hkv][d]
     (innermost dim contiguous, K and V with equal strides), prefix_len [B],
-    parent [B][T], n_nodes [B] or None.  Returns (out, lse, sel_blocks)."""
+    parent [B][T], n_nodes [B] or None.  prefix_only: the partial over the
+    prefix keys alone (a rank's slice of a split prefix).  Returns
+    (out, lse, sel_blocks)."""
     dev = _need_cuda(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent, n_nodes, k_block_mean)
     if q.dtype == torch.bfloat16:
         dt = TV_BF16
@@ -237,7 +246,7 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent, n_
                  parent.data_ptr(), parent.stride(0),
                  _ptr(n_nodes), float(scale), int(sparse_topk), int(block_size), _ptr(k_block_mean),
                  out.data_ptr(), out.stride(0), out.stride(1), out.stride(2),
-                 _ptr(lse), _ptr(sel_blocks), _ptr(dev_status))
+                 _ptr(lse), _ptr(sel_blocks), _ptr(dev_status), int(bool(prefix_only)))
     L = lib()
     global last_attn_path, last_attn_launches
     last_attn_path = L.tv_attn_path(ctypes.byref(a))
@@ -247,6 +256,34 @@ def tree_verify_attn(q, k_cache, v_cache, prefix_len, k_tree, v_tree, parent, n_
     ws = _workspace(dev, sh, need)
     _check(L.tree_verify_attn(ctypes.byref(a), _aligned_ptr(ws), need, sh), "tree_verify_attn")
     return out, lse, sel_blocks
+
+
+def tree_verify_attn_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
+    """Log-sum-exp merge of N attention partials over disjoint key sets
+    (include/tree_verify.h, tree_verify_attn_merge): o_parts [N][B][T][Hq][d]
+    bf16/fp32, lse_parts [N][B][T][Hq] fp32, both contiguous.  Returns
+    (out [B][T][Hq][d], lse [B][T][Hq])."""
+    _need_cuda(o_parts, lse_parts, out, lse)
+    if o_parts.dtype == torch.bfloat16:
+        dt = TV_BF16
+    elif o_parts.dtype == torch.float32:
+        dt = TV_FP32
+    else:
+        raise TVError("o_parts must be bf16 or fp32")
+    if not o_parts.is_contiguous() or not lse_parts.is_contiguous() or lse_parts.dtype != torch.float32:
+        raise TVError("o_parts and lse_parts must be contiguous; lse_parts fp32")
+    N, B, T, Hq, d = o_parts.shape
+    if tuple(lse_parts.shape) != (N, B, T, Hq):
+        raise TVError("lse_parts must be [N][B][T][Hq]")
+    if out is None:
+        out = torch.empty(B, T, Hq, d, dtype=o_parts.dtype, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty(B, T, Hq, dtype=torch.float32, device=o_parts.device)
+    if not out.is_contiguous() or out.dtype != o_parts.dtype or not lse.is_contiguous():
+        raise TVError("out must be contiguous with o_parts' dtype; lse contiguous fp32")
+    a = AttnMergeArgs(dt, N, B, T, Hq, d, o_parts.data_ptr(), lse_parts.data_ptr(), out.data_ptr(), lse.data_ptr())
+    _check(lib().tree_verify_attn_merge(ctypes.byref(a), _stream(stream)), "tree_verify_attn_merge")
+    return out, lse
 
 
 # Which attention kernels the last tree_verify_attn call ran (tv_attn_path).

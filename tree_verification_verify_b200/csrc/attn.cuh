@@ -19,6 +19,7 @@ struct AttnParams {
   void* out; int64_t o_sb, o_st, o_sh;
   float* lse;
   uint32_t* status;
+  int prefix_only;             // partial over the prefix keys alone (no tree keys)
   // block top-k
   int topk, block_size, nblk_max;
   const float* kbar;           // [B][nblk_max][Hkv][d] (caller's or workspace)

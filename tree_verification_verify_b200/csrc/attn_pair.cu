@@ -163,7 +163,9 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
   const int nodes_b = max(0, min(NT, n - i0 - NT));
   const int nq = nodes_b > 0 ? 2 : 1;      // query tiles with rows
   const int nodes_here = nodes_a + nodes_b;
-  const bool has_tree = (chunk == C - 1);   // the last chunk is the shortest
+  // the last chunk (the shortest) also runs the tree tiles, unless the call
+  // is a prefix-only partial
+  const bool has_tree = (chunk == C - 1) && !p.prefix_only;
   // softmax threads: tile qt = warp / 4, row = TMEM lane = tid % 128
   const int qt = (warp >> 2) & 1;
   const int row = tid & (kRows - 1);
@@ -592,7 +594,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
     ep_lse2 = lse2;
     ep_inv = inv;
     if (row_valid && has_tree && !my_ok) set_status(p.status, TV_DEV_BAD_PARENT);
-    if (bad_len && has_tree && qt == 0 && row == 0) set_status(p.status, TV_DEV_BAD_LEN);
+    if (bad_len && chunk == C - 1 && qt == 0 && row == 0) set_status(p.status, TV_DEV_BAD_LEN);
   }
 
   // ------------------------------------------------------------ cluster merge
@@ -684,6 +686,9 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
             acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
           }
         }
+        // no keys at all (an empty slice of a prefix-only partial): O = 0,
+        // lse = -inf
+        const bool empty = !bad && den == 0.f;
         const bool okr = !bad && den > 0.f;
         const float iv = okr ? 1.f / den : 0.f;
         uint2 wv;
@@ -691,14 +696,14 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
           wv.x = pack_bf16(acc.x * iv, acc.y * iv);
           wv.y = pack_bf16(acc.z * iv, acc.w * iv);
         } else {
-          wv.x = wv.y = pack_bf16(NAN, NAN);
+          wv.x = wv.y = empty ? 0u : pack_bf16(NAN, NAN);
         }
         const int node = i0 + r * NT + t / G, head = g * G + t % G;
         __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + node * p.o_st + head * p.o_sh;
         *reinterpret_cast<uint2*>(o + lane * 4) = wv;
         if (lane == 0 && p.lse)
           p.lse[(static_cast<int64_t>(b) * p.T + node) * p.Hq + head] =
-              okr ? (M + __log2f(den)) * 0.6931471805599453f : NAN;
+              okr ? (M + __log2f(den)) * 0.6931471805599453f : (empty ? -INFINITY : NAN);
       }
     }
     fence_before();

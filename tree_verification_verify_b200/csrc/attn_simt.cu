@@ -151,6 +151,16 @@ attn_tree_kernel(AttnParams p) {
   const int n = p.n_nodes ? p.n_nodes[b] : p.T;
   if (n < 0 || n > p.T || i >= n) return;
   const int32_t* par = p.parent + b * p.par_sb;
+  if (p.prefix_only) {
+    // a prefix-only partial: no tree keys (parent[] is not read)
+    if (threadIdx.x == 0 && g == 0) p.node_ok[static_cast<int64_t>(b) * p.T + i] = 1;
+    for (int hg = warp; hg < p.G; hg += kTreeWarps) {
+      const int64_t pr = part_row(p, p.nchunk, b, i, g * p.G + hg);
+      for (int k = lane; k < D; k += 32) p.part_o[pr * D + k] = 0.f;
+      if (lane == 0) p.part_lse[pr] = -INFINITY;
+    }
+    return;
+  }
   if (threadIdx.x == 0) {
     // root path of node i (i first, root last); malformed chains stop early
     int len = 0, ok = (par[0] == -1) ? 1 : 0;
@@ -276,10 +286,56 @@ attn_merge_kernel(AttnParams p) {
 #pragma unroll
     for (int k = 0; k < DL; ++k) acc[k] = fmaf(w, p.part_o[pr * D + lane + 32 * k], acc[k]);
   }
-  const float inv = 1.f / den;
+  // no keys at all (an empty slice of a prefix-only partial): O = 0, lse = -inf
+  const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
   for (int k = 0; k < DL; ++k) o[lane + 32 * k] = static_cast<T>(acc[k] * inv);
-  if (p.lse && lane == 0) p.lse[row] = M + logf(den);
+  if (p.lse && lane == 0) p.lse[row] = den > 0.f ? M + logf(den) : -INFINITY;
+}
+
+// Log-sum-exp merge of N stacked partials (tree_verify_attn_merge): one
+// warp per output row.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+attn_partial_merge_kernel(const T* __restrict__ o_parts, const float* __restrict__ lse_parts, T* out, float* lse,
+                          int N, int64_t nrows) {
+  constexpr int DL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= nrows) return;
+  float lc = -INFINITY;
+  bool bad = false;
+  for (int c = lane; c < N; c += 32) {
+    const float v = lse_parts[static_cast<int64_t>(c) * nrows + row];
+    bad |= (v != v);
+    lc = fmaxf(lc, v);
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  const float M = warp_max(lc);
+  float wsum = 0.f;
+  for (int c = lane; c < N; c += 32) {
+    const float v = lse_parts[static_cast<int64_t>(c) * nrows + row];
+    wsum += (v > -INFINITY) ? expf(v - M) : 0.f;
+  }
+  const float den = warp_sumf(wsum);
+  float acc[DL];
+#pragma unroll
+  for (int k = 0; k < DL; ++k) acc[k] = 0.f;
+  if (!bad && den > 0.f) {
+    for (int c = 0; c < N; ++c) {
+      const float v = lse_parts[static_cast<int64_t>(c) * nrows + row];
+      if (!(v > -INFINITY)) continue;
+      const float w = expf(v - M);
+      const T* src = o_parts + (static_cast<int64_t>(c) * nrows + row) * D;
+#pragma unroll
+      for (int k = 0; k < DL; ++k) acc[k] = fmaf(w, to_f32(src[lane + 32 * k]), acc[k]);
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  T* dst = out + row * D;
+#pragma unroll
+  for (int k = 0; k < DL; ++k) dst[lane + 32 * k] = static_cast<T>(bad ? NAN : acc[k] * inv);
+  if (lse && lane == 0) lse[row] = bad ? NAN : (den > 0.f ? M + logf(den) : -INFINITY);
 }
 
 // ------------------------------------------------------------ launchers
@@ -339,6 +395,26 @@ cudaError_t launch_attn_tree(const AttnParams& p, cudaStream_t s) {
 cudaError_t launch_attn_merge(const AttnParams& p, cudaStream_t s) {
   if (p.dtype == TV_BF16) { TV_DISPATCH_D(launch_merge_t, __nv_bfloat16, p, s) }
   TV_DISPATCH_D(launch_merge_t, float, p, s)
+}
+
+template <typename T, int D>
+static cudaError_t launch_partial_merge_t(const tv_attn_merge_args* a, cudaStream_t s) {
+  const int64_t nrows = static_cast<int64_t>(a->B) * a->T * a->Hq;
+  const int64_t blocks = (nrows + 7) / 8;
+  attn_partial_merge_kernel<T, D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      static_cast<const T*>(a->o_parts), a->lse_parts, static_cast<T*>(a->out), a->lse, a->N, nrows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_partial_merge(const tv_attn_merge_args* a, cudaStream_t s) {
+  if (a->dtype == TV_BF16) {
+    if (a->d == 128) return launch_partial_merge_t<__nv_bfloat16, 128>(a, s);
+    if (a->d == 64) return launch_partial_merge_t<__nv_bfloat16, 64>(a, s);
+    return launch_partial_merge_t<__nv_bfloat16, 32>(a, s);
+  }
+  if (a->d == 128) return launch_partial_merge_t<float, 128>(a, s);
+  if (a->d == 64) return launch_partial_merge_t<float, 64>(a, s);
+  return launch_partial_merge_t<float, 32>(a, s);
 }
 
 }  // namespace tv

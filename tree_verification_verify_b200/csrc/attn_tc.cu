@@ -172,7 +172,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   // kept blocks is listed (block top-k)
   int nprefix = SPARSE ? 0 : ((k1 > k0) ? (k1 - k0 + kKeys - 1) / kKeys : 0);
   const int nodes_here = min(kRows / G, n - i0);
-  const bool has_tree = (chunk == C - 1);   // the last chunk is the shortest
+  // the last chunk (the shortest) also runs the tree tiles, unless the call
+  // is a prefix-only partial
+  const bool has_tree = (chunk == C - 1) && !p.prefix_only;
   // this thread's query row (softmax warps)
   // softmax threads: query row tid % 128 (TMEM lane), column half tid / 128
   const int row = tid & (kRows - 1);
@@ -739,7 +741,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     // the stage is read by bulk copies (async proxy)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (half == 0 && row_valid && has_tree && !my_ok) set_status(p.status, TV_DEV_BAD_PARENT);
-    if (bad_len && has_tree && tid == 0) set_status(p.status, TV_DEV_BAD_LEN);
+    if (bad_len && chunk == C - 1 && tid == 0) set_status(p.status, TV_DEV_BAD_LEN);
   }
 
   // ------------------------------------------------------------ cluster merge
@@ -804,6 +806,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
         }
       }
+      // no keys at all (an empty slice of a prefix-only partial): O = 0,
+      // lse = -inf
+      const bool empty = !bad && den == 0.f;
       const bool okr = !bad && den > 0.f;
       const float iv = okr ? 1.f / den : 0.f;
       uint2 wv;
@@ -811,14 +816,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         wv.x = pack_bf16(acc.x * iv, acc.y * iv);
         wv.y = pack_bf16(acc.z * iv, acc.w * iv);
       } else {
-        wv.x = wv.y = pack_bf16(NAN, NAN);
+        wv.x = wv.y = empty ? 0u : pack_bf16(NAN, NAN);
       }
       const int node = i0 + t / G, head = g * G + t % G;
       __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + node * p.o_st + head * p.o_sh;
       *reinterpret_cast<uint2*>(o + lane * 4) = wv;
       if (lane == 0 && p.lse)
         p.lse[(static_cast<int64_t>(b) * p.T + node) * p.Hq + head] =
-            okr ? (M + __log2f(den)) * 0.6931471805599453f : NAN;
+            okr ? (M + __log2f(den)) * 0.6931471805599453f : (empty ? -INFINITY : NAN);
     }
   }
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");

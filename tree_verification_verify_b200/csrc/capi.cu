@@ -24,6 +24,7 @@ cudaError_t launch_block_select(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attn_sparse(const AttnParams& p, cudaStream_t stream);
 int num_sms();
 cudaError_t launch_commit(const tv_commit_args* a, cudaStream_t stream);
+cudaError_t launch_attn_partial_merge(const tv_attn_merge_args* a, cudaStream_t stream);
 }  // namespace tv
 
 using namespace tv;
@@ -58,6 +59,8 @@ tv_status check_attn(const tv_attn_args* a) {
   if (!(a->scale >= 0.f) || !std::isfinite(a->scale)) return TV_ERR_INVALID_ARG;
   if (a->sparse_topk < 0) return TV_ERR_INVALID_ARG;
   if (a->sparse_topk > 0 && a->block_size <= 0) return TV_ERR_INVALID_ARG;
+  if (a->prefix_only != 0 && a->prefix_only != 1) return TV_ERR_INVALID_ARG;
+  if (a->prefix_only && a->sparse_topk > 0) return TV_ERR_UNSUPPORTED;
   if (a->d != 32 && a->d != 64 && a->d != 128) return TV_ERR_UNSUPPORTED;
   if (a->Hq / a->Hkv > 64) return TV_ERR_UNSUPPORTED;
   if (a->B > 0 && a->T > 0) {
@@ -204,6 +207,7 @@ extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws
   p.out = a->out; p.o_sb = a->o_sb; p.o_st = a->o_st; p.o_sh = a->o_sh;
   p.lse = a->lse;
   p.status = a->dev_status;
+  p.prefix_only = a->prefix_only;
   p.nchunk = pl.nchunk; p.chunk_len = pl.chunk_len; p.node_tile = pl.node_tile;
   unsigned char* w = static_cast<unsigned char*>(ws);
   p.part_o = reinterpret_cast<float*>(w + pl.off_o);
@@ -241,6 +245,17 @@ extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws
   if (e != cudaSuccess) return from_cuda(e);
   e = launch_attn_merge(p, s);
   return from_cuda(e);
+}
+
+extern "C" tv_status tree_verify_attn_merge(const tv_attn_merge_args* a, tv_stream_t stream) {
+  if (!a) return TV_ERR_INVALID_ARG;
+  if (a->dtype != TV_FP32 && a->dtype != TV_BF16) return TV_ERR_INVALID_ARG;
+  if (a->N < 1 || a->B < 0 || a->T < 0 || a->Hq < 0) return TV_ERR_INVALID_ARG;
+  if (a->N > 64) return TV_ERR_UNSUPPORTED;
+  if (a->d != 32 && a->d != 64 && a->d != 128) return TV_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(a->B) * a->T * a->Hq == 0) return TV_OK;
+  if (!a->o_parts || !a->lse_parts || !a->out) return TV_ERR_INVALID_ARG;
+  return from_cuda(launch_attn_partial_merge(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 // ------------------------------------------------------------ acceptance
