@@ -414,6 +414,23 @@ TV_API tv_status tv_philox_uniforms(uint64_t seed, uint64_t step, const int32_t*
                              const int32_t* node, const int32_t* draw,
                              const int32_t* tag, double* out, int32_t n,
                              tv_stream_t stream);
+/* The exponential behind tree_expand_topb's fp64 log-sum-exp of a row (a
+ * table-driven method: Tang, ACM TOMS 15(2), 1989), for checking it:
+ * out[k] = e^(t[k]) for -700 <= t[k] <= 0, 0 for t[k] < -700 (such terms
+ * are below 1e-300 of a row's largest, which contributes 1).  t and out
+ * are device memory of n entries; t[k] > 0 is not supported (out[k] is
+ * then unspecified). */
+TV_API tv_status tv_expand_exp(const double* t, double* out, int32_t n, tv_stream_t stream);
+/* Test hook for the bounded waits of tree_expand_topb.  With polls > 0,
+ * every row staged in shared memory (rows 16-byte aligned with a row stride
+ * of a multiple of 4 elements, V*4 bytes small enough) waits for its first
+ * chunk as if that copy were lost: `polls` non-blocking tests of a barrier
+ * phase that nothing completes.  The wait expires, the row's real copies
+ * are drained (bounded wait), the row is dropped (its node counts as
+ * expanded, with no children) and TV_DEV_TIMEOUT is set in dev_status.
+ * polls = 0 restores normal waits.  Applies to the current device,
+ * synchronously; not for use while expansion calls are in flight. */
+TV_API tv_status tv_expand_set_wait_limit(uint32_t polls);
 
 #ifdef __cplusplus
 }

@@ -249,3 +249,55 @@ def test_beam_mode_keeps_less_mass_than_best_first():
     print(f"expected accepted length (sum of path probabilities): best-first {mass['bestfirst']:.3f}, "
           f"beam {mass['beam']:.3f}")
     assert mass["bestfirst"] > mass["beam"]
+
+
+def test_row_exponential_error_bound():
+    """The fp64 exponential of the row pass's log-sum-exp (a table-driven
+    method: 256-entry table of 2^(j/256), degree-4 Taylor remainder on
+    |r| <= ln2/512) against numpy's exp: within 4 ulp over [-700, 0],
+    including the reduction boundaries; 0 below -700."""
+    import tree_verification_verify_b200 as tv
+    rng = np.random.default_rng(0)
+    step = math.log(2.0) / 256.0
+    t = np.concatenate([
+        -rng.uniform(0.0, 700.0, 200000),
+        -rng.uniform(0.0, 1.0, 100000),
+        -np.arange(0, 2000) * step,                      # reduction grid points
+        -(np.arange(0, 2000) + 0.5) * step,              # half-way points
+        -(np.arange(0, 2000) + 0.5) * step * (1 + 1e-15),
+        np.array([0.0, -0.0, -1e-300, -1e-17, -700.0, -699.999999]),
+    ])
+    got = tv.expand_exp(torch.tensor(t, dtype=torch.float64, device="cuda")).cpu().numpy()
+    want = np.exp(t)
+    rel = np.abs(got - want) / want
+    print(f"max relative error {rel.max():.3e} ({rel.max() / 2.0 ** -52:.2f} ulp)")
+    assert rel.max() <= 4 * 2.0 ** -52
+    low = tv.expand_exp(torch.tensor([-700.5, -800.0, -1e300, -math.inf], dtype=torch.float64,
+                                     device="cuda")).cpu().numpy()
+    assert np.all(low == 0.0)
+
+
+def test_row_wait_timeout_status():
+    """A bounded wait that runs out (the test hook makes a staged row wait
+    for a copy phase that nothing completes): the row is dropped after its
+    real copies land, TV_DEV_TIMEOUT is set, nothing is appended, and the
+    context stays usable for a normal round afterwards."""
+    import tree_verification_verify_b200 as tv
+    V, Bsel, budget = 32000, 16, 64
+    z = torch.randn(1, V, device="cuda")
+    root = torch.zeros(1, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = tv.tree_expand_init(budget, V, Bsel)
+    try:
+        tv.expand_set_wait_limit(64)
+        tv.tree_expand_topb(st, z, root, dev_status=status)
+        torch.cuda.synchronize()
+    finally:
+        tv.expand_set_wait_limit(0)
+    assert int(status.item()) & 32, int(status.item())
+    assert int(st.n_appended.item()) == 0 and int(st.n_nodes.item()) == 1
+    status.zero_()
+    st2 = tv.tree_expand_init(budget, V, Bsel)
+    tv.tree_expand_topb(st2, z, root, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0 and int(st2.n_appended.item()) == Bsel

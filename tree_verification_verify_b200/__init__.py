@@ -110,7 +110,9 @@ def lib() -> ctypes.CDLL:
                            ("tree_expand_topb", [ctypes.POINTER(ExpandArgs), c_vp, c_size, c_vp]),
                            ("tree_expand_init", [ctypes.POINTER(ExpandArgs), c_i32, c_vp]),
                            ("tree_commit_kv", [ctypes.POINTER(CommitArgs), c_vp]),
-                           ("tv_philox_uniforms", [c_u64, c_u64, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp])):
+                           ("tv_philox_uniforms", [c_u64, c_u64, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp]),
+                           ("tv_expand_exp", [c_vp, c_vp, c_i32, c_vp]),
+                           ("tv_expand_set_wait_limit", [ctypes.c_uint32])):
             f = getattr(L, name)
             f.argtypes = args
             f.restype = ctypes.c_int
@@ -489,4 +491,21 @@ def philox_uniforms(seed: int, step: int, b, node, draw, tag, stream=None) -> to
                                     b.data_ptr(), node.data_ptr(), draw.data_ptr(), tag.data_ptr(),
                                     out.data_ptr(), b.numel(), _stream(stream)), "tv_philox_uniforms")
     return out
+
+
+def expand_exp(t, stream=None) -> torch.Tensor:
+    """The exponential of tree_expand_topb's fp64 log-sum-exp (tv_expand_exp):
+    e^t for fp64 device t <= 0 (0 below -700)."""
+    dev = _need_cuda(t)
+    if t.dtype != torch.float64 or not t.is_contiguous():
+        raise TVError("t must be contiguous fp64")
+    out = torch.empty_like(t)
+    _check(lib().tv_expand_exp(t.data_ptr(), out.data_ptr(), t.numel(), _stream(stream)), "tv_expand_exp")
+    return out
+
+
+def expand_set_wait_limit(polls: int) -> None:
+    """Test hook (tv_expand_set_wait_limit): at most `polls` non-blocking
+    tests per staged chunk in tree_expand_topb's row pass (0: default)."""
+    _check(lib().tv_expand_set_wait_limit(int(polls)), "tv_expand_set_wait_limit")
 

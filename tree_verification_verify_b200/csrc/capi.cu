@@ -13,6 +13,8 @@ cudaError_t launch_accept(const tv_accept_args* a, int mode, void* ws, cudaStrea
 size_t expand_pool_bytes(int budget, int V);
 cudaError_t launch_expand_init(const tv_expand_args* a, int root_token, cudaStream_t stream);
 cudaError_t launch_expand(const tv_expand_args* a, cudaStream_t stream);
+cudaError_t launch_expand_exp(const double* t, double* out, int n, cudaStream_t stream);
+cudaError_t expand_set_wait_limit(uint32_t polls);
 bool attn_tc_supported(const tv_attn_args* a);
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream);
 int attn_tc_active_clusters(int c);
@@ -405,6 +407,17 @@ extern "C" tv_status tv_philox_uniforms(uint64_t seed, uint64_t step, const int3
   philox_uniforms_kernel<<<(n + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       seed, step, b, node, draw, tag, out, n);
   return from_cuda(cudaGetLastError());
+}
+
+extern "C" tv_status tv_expand_set_wait_limit(uint32_t polls) {
+  return from_cuda(tv::expand_set_wait_limit(polls));
+}
+
+extern "C" tv_status tv_expand_exp(const double* t, double* out, int32_t n, tv_stream_t stream) {
+  if (n < 0) return TV_ERR_INVALID_ARG;
+  if (n == 0) return TV_OK;
+  if (!t || !out) return TV_ERR_INVALID_ARG;
+  return from_cuda(tv::launch_expand_exp(t, out, n, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 extern "C" const char* tree_verify_version(void) { return "treeverify 0.1.0 sm_100a"; }

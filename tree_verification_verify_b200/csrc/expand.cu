@@ -39,6 +39,11 @@
 
 namespace tv {
 
+// Test hook (tv_expand_set_wait_limit): when nonzero, a staged row waits
+// for its first chunk with this many non-blocking tests of a barrier that
+// nothing arrives on (as if the copy were lost), so the wait expires.
+__device__ uint32_t g_row_wait_polls = 0u;
+
 struct NodeMeta {
   int32_t len;        // entries in the node's sorted list (0: not expanded)
   int32_t cursor;     // first entry not yet taken
@@ -117,6 +122,7 @@ struct ExpandShared {
   uint32_t boff[kBins];
   uint32_t bfill[kBins];
   uint64_t bar[kMaxChunks];
+  uint64_t lost_bar;  // never arrived on (the wait-expiry test hook)
   double etab[256];   // 2^(j/256)
   double red_d[kWarps];
   float red_f[kWarps];
@@ -692,6 +698,7 @@ __device__ void row_body(const ExpandParams& p, int r, unsigned char* dsm, Expan
   if (staged && tid == 0) {
     sh.abort = 0;
     for (int c = 0; c < ncopy; ++c) tc::mbar_init(&sh.bar[c], 1);
+    tc::mbar_init(&sh.lost_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     for (; issued < ncopy; ++issued) {
@@ -754,9 +761,19 @@ __device__ void row_body(const ExpandParams& p, int r, unsigned char* dsm, Expan
   bool ok = true;
 
   // one lane per warp waits for a staged chunk (the warp then reads it)
+  const uint32_t lost = g_row_wait_polls;
   auto wait_chunk = [&](int c) {
     bool w = true;
-    if (lane == 0) w = tc::mbar_wait(&sh.bar[c], 0, &sh.abort);
+    if (lane == 0) {
+      if (c == 0 && lost != 0u) {
+        // the test hook: the first phase of a barrier nothing arrives on
+        w = false;
+        for (uint32_t it = 0; it < lost && !w; ++it) w = tc::mbar_test(&sh.lost_bar, 0);
+        if (!w) sh.abort = 1;
+      } else {
+        w = tc::mbar_wait(&sh.bar[c], 0, &sh.abort);
+      }
+    }
     __syncwarp();
     return __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
   };
@@ -1476,6 +1493,14 @@ __global__ void expand_init_kernel(ExpandParams p, int root_token) {
   }
 }
 
+__global__ void expand_exp_kernel(const double* t, double* out, int n) {
+  __shared__ double T[256];
+  for (int j = threadIdx.x; j < 256; j += blockDim.x) T[j] = exp2(static_cast<double>(j) * (1.0 / 256.0));
+  __syncthreads();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = exp_neg(t[i], T);
+}
+
 // ------------------------------------------------------------ host side
 
 size_t expand_pool_bytes(int budget, int V) {
@@ -1500,6 +1525,15 @@ static ExpandParams make_params(const tv_expand_args* a) {
   p.frontier = a->frontier; p.n_appended = a->n_appended;
   p.status = a->dev_status;
   return p;
+}
+
+cudaError_t expand_set_wait_limit(uint32_t polls) {
+  return cudaMemcpyToSymbol(g_row_wait_polls, &polls, sizeof(polls));
+}
+
+cudaError_t launch_expand_exp(const double* t, double* out, int n, cudaStream_t stream) {
+  expand_exp_kernel<<<(n + 255) / 256, 256, 0, stream>>>(t, out, n);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_expand_init(const tv_expand_args* a, int root_token, cudaStream_t stream) {
