@@ -75,7 +75,7 @@ KERNEL_SOURCES = {
     "accept_node_kernel": "tree_verification_verify_b200/csrc/accept.cu",
     "attn_tc_kernel": "tree_verification_verify_b200/csrc/attn_tc.cu",
     "attn_pair_kernel": "tree_verification_verify_b200/csrc/attn_pair.cu",
-    "expand_rows_kernel": "tree_verification_verify_b200/csrc/expand.cu",
+    "expand_round_kernel": "tree_verification_verify_b200/csrc/expand.cu",
 }
 
 
@@ -378,7 +378,7 @@ class Step:
 
     def launches_per_step(self):
         attn = self.attn_launches
-        exp = (1 + 2 * len(self.exp_logits)) if self.expand else 0
+        exp = (1 + len(self.exp_logits)) if self.expand else 0
         return attn + 1 + exp
 
     def near_threshold(self):
@@ -1081,10 +1081,10 @@ def main_roofline(step, ms, hbm, bf16, src):
     exp_s = ms.get("expand", 0.0) * 1e-3
     if exp_s >= max(acc_s, attn_s):
         achieved = step.expand_bytes / exp_s / 1e9
-        roof = {"kernel": "tree_expand_topb (16 rounds: row + merge launches)", "bound": "hbm",
+        roof = {"kernel": "tree_expand_topb (16 rounds, one launch each)", "bound": "hbm",
                 "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
                 "algorithmic_bytes": step.expand_bytes, "units": "draft logit rows of all rounds x V x 4 B"}
-        tk = "expand_rows_kernel"
+        tk = "expand_round_kernel"
     elif acc_s >= attn_s:
         achieved = step.accept_bytes / acc_s / 1e9
         roof = {"kernel": "accept_node_kernel (tree_accept: one launch)", "bound": "hbm",

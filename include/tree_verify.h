@@ -391,7 +391,12 @@ TV_API tv_status tree_commit_kv(const tv_commit_args* a, tv_stream_t stream);
  * the tensor-core kernel (bf16, d = 128, blocks of 64, G >= 4),
  * 4 = the tcgen05 kernel in its two-query-tile form (each CTA takes two
  * 128-row tiles of packed (node, head) rows that share every K/V tile;
- * chosen by the same cost model as 1, for long prefixes),
+ * chosen by the same cost model as 1, for long prefixes; the prefix chunks
+ * of a tile pair form a thread-block cluster and merge on chip),
+ * 5 = the same two-query-tile kernel with up to 16 prefix chunks per tile
+ * pair merged through the workspace (no cluster: the planner's choice when
+ * more chunks than a cluster fills the GPU better; the workspace holds the
+ * chunks' fp32 rows),
  * -1 = the arguments are rejected. */
 TV_API int32_t tv_attn_path(const tv_attn_args* a);
 /* How many kernels tree_verify_attn launches for these arguments (0 when

@@ -42,7 +42,8 @@ def _slice(case, lo, hi, dev="cuda"):
 
 @pytest.mark.parametrize("B,T,Hq,Hkv,d,L,dtype,paths", [
     (2, 40, 32, 8, 128, [1000, 0], "bf16", (1,)),           # one-tile tensor-core kernel
-    (1, 256, 32, 8, 128, [32768], "bf16", (4,)),            # two-tile tensor-core kernel
+    (1, 256, 32, 8, 128, [32768], "bf16", (4, 5)),          # two-tile tensor-core kernel
+    (1, 256, 32, 8, 128, [65536], "bf16", (5,)),            # ... chunks merged through the workspace
     (2, 17, 8, 2, 64, [300, 0], "fp32", (0,)),              # CUDA cores
 ])
 def test_prefix_only_partial(B, T, Hq, Hkv, d, L, dtype, paths):

@@ -292,7 +292,8 @@ def tree_verify_attn_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
 last_attn_path = None
 last_attn_launches = None
 ATTN_PATHS = {0: "cuda-core split-KV", 1: "tcgen05 prefix", 2: "block top-k sparse (cuda cores)",
-              3: "block top-k sparse (tcgen05)", 4: "tcgen05 prefix, two query tiles per CTA"}
+              3: "block top-k sparse (tcgen05)", 4: "tcgen05 prefix, two query tiles per CTA",
+              5: "tcgen05 prefix, two query tiles per CTA, chunks merged through the workspace"}
 
 
 # --------------------------------------------------------------- KV commit

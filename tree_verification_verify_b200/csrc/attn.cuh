@@ -20,6 +20,8 @@ struct AttnParams {
   float* lse;
   uint32_t* status;
   int prefix_only;             // partial over the prefix keys alone (no tree keys)
+  int gmerge;                  // two-tile kernel: chunks merged through the workspace
+                               // (part_o [unit][chunk][2][128][d], part_lse [unit][chunk][2][128])
   // block top-k
   int topk, block_size, nblk_max;
   const float* kbar;           // [B][nblk_max][Hkv][d] (caller's or workspace)

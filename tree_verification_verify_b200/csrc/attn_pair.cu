@@ -20,7 +20,10 @@
 // the union U of the root paths of both tiles' nodes, gathered into K/V
 // tiles and masked per row by the row's ancestors in U.  At the end the
 // chunks' normalised O rows and log-sum-exps are merged over distributed
-// shared memory, tile A then tile B.
+// shared memory, tile A then tile B; or, when the planner splits a pair into
+// more chunks than a cluster holds at once, through the workspace: every
+// chunk writes its normalised fp32 rows and log-sum-exps to its slot, and
+// the last chunk of the pair to finish (a ticket) merges them.
 //
 // Warp roles (384 threads):
 //   warps 0-3  softmax / correction / epilogue of tile A: thread t owns row
@@ -63,7 +66,8 @@ constexpr int kD = 128;
 constexpr int kKS = 2;              // K ring stages
 constexpr int kVS = 2;              // V ring stages
 constexpr int kMaxT = 2048;         // tree nodes handled by this kernel
-constexpr int kMaxCluster = 8;      // chunks per tile pair
+constexpr int kMaxCluster = 8;      // chunks per tile pair merged over distributed shared memory
+constexpr int kMaxChunksGlobal = 16;  // chunks per tile pair merged through the workspace
 constexpr uint32_t kHalfBytes = kRows * 128;            // 128 rows x 128 B
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;         // 32 KB (d = 128 bf16)
 constexpr uint32_t kSmemQ = 0;                            // Q_A, Q_B
@@ -98,6 +102,7 @@ struct Bars {
   uint64_t inbox_full;              // merge round r: phase r
   uint32_t tmem_base;
   int abort;
+  int last;                         // workspace merge: this CTA merges the pair's chunks
   int nU;                           // nodes in the union of root paths
   uint32_t bm[kMaxT / 32];          // node bitmap of U
   int pre[kMaxT / 32];              // marked nodes below each bitmap word
@@ -209,7 +214,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     // the bytes the cluster will copy into this CTA's inbox in round 0
-    mbar_expect_tx(&bars.inbox_full, static_cast<uint32_t>(C) * merge_bytes(own_rows(0)));
+    if (!p.gmerge) mbar_expect_tx(&bars.inbox_full, static_cast<uint32_t>(C) * merge_bytes(own_rows(0)));
   }
   if (warp == kWarpMma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -597,6 +602,91 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
     if (bad_len && chunk == C - 1 && qt == 0 && row == 0) set_status(p.status, TV_DEV_BAD_LEN);
   }
 
+  if (p.gmerge) {
+    // ---------------------------------------------------------- workspace merge
+    // Slot (unit, chunk) holds the chunk's normalised fp32 O rows of both
+    // tiles and their log2-sum-exp; the last chunk to finish merges.
+    const int unit = static_cast<int>(blockIdx.z) * static_cast<int>(gridDim.y) + pair;
+    fence_before();
+    __syncthreads();
+    fence_after();
+    if (warp < 8 && qt < nq) {
+      const float inv = ep_inv;
+      const bool have = inv > 0.f;
+      float* dst = p.part_o + ((static_cast<int64_t>(unit) * C + chunk) * 2 + qt) * kRows * kD +
+                   static_cast<int64_t>(row) * kD;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + col_o(qt) + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          __stcg(reinterpret_cast<float4*>(dst + c * 32 + 4 * q),
+                 have ? make_float4(v[4 * q] * inv, v[4 * q + 1] * inv, v[4 * q + 2] * inv, v[4 * q + 3] * inv)
+                      : make_float4(0.f, 0.f, 0.f, 0.f));
+      }
+      __stcg(p.part_lse + ((static_cast<int64_t>(unit) * C + chunk) * 2 + qt) * kRows + row, ep_lse2);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      const int t = atomicAdd(&p.tickets[unit], 1);
+      bars.last = (t == C - 1) ? 1 : 0;
+      if (bars.last) {
+        __threadfence();
+        p.tickets[unit] = 0;                   // ready for the next call
+      }
+    }
+    __syncthreads();
+    if (bars.last) {
+      for (int r = 0; r < nq; ++r) {
+        const int rows_r = (r ? nodes_b : nodes_a) * G;
+        for (int t = warp; t < rows_r; t += kThreads / 32) {
+          const float* ls = p.part_lse + static_cast<int64_t>(unit) * C * 2 * kRows + r * kRows + t;
+          float M = -INFINITY;
+          bool bad = false;
+          for (int c = 0; c < C; ++c) {
+            const float lc = __ldcg(ls + c * 2 * kRows);
+            bad |= (lc != lc);
+            M = fmaxf(M, lc);
+          }
+          float den = 0.f;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int c = 0; c < C; ++c) {
+            const float lc = __ldcg(ls + c * 2 * kRows);
+            const float w = (lc > -INFINITY) ? ex2_approx(lc - M) : 0.f;
+            den += w;
+            if (w != 0.f) {
+              const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                  p.part_o + ((static_cast<int64_t>(unit) * C + c) * 2 + r) * kRows * kD +
+                  static_cast<int64_t>(t) * kD + lane * 4));
+              acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+              acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+            }
+          }
+          // no keys at all (an empty slice of a prefix-only partial): O = 0,
+          // lse = -inf
+          const bool empty = !bad && den == 0.f;
+          const bool okr = !bad && den > 0.f;
+          const float iv = okr ? 1.f / den : 0.f;
+          uint2 wv;
+          if (okr) {
+            wv.x = pack_bf16(acc.x * iv, acc.y * iv);
+            wv.y = pack_bf16(acc.z * iv, acc.w * iv);
+          } else {
+            wv.x = wv.y = empty ? 0u : pack_bf16(NAN, NAN);
+          }
+          const int node = i0 + r * NT + t / G, head = g * G + t % G;
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + b * p.o_sb + node * p.o_st + head * p.o_sh;
+          *reinterpret_cast<uint2*>(o + lane * 4) = wv;
+          if (lane == 0 && p.lse)
+            p.lse[(static_cast<int64_t>(b) * p.T + node) * p.Hq + head] =
+                okr ? (M + __log2f(den)) * 0.6931471805599453f : (empty ? -INFINITY : NAN);
+        }
+      }
+    }
+  } else {
   // ------------------------------------------------------------ cluster merge
   // One round per query tile.  Each CTA stages its normalised fp32 O rows of
   // the tile (the idle V ring) and their log2-sum-exp; once every CTA has
@@ -710,6 +800,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
     cl.sync();                  // every copy out of every stage has landed; inboxes consumed
     fence_after();
   }
+  }
   if (warp == kWarpMma) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
@@ -753,7 +844,8 @@ int attn_pair_active_clusters(int c) {
 cudaError_t launch_attn_pair(const AttnParams& p, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   const int G = p.G;
-  if (p.nchunk < 1 || p.nchunk > kMaxCluster || p.T > kMaxT || p.d != kD) return cudaErrorInvalidValue;
+  if (p.nchunk < 1 || p.nchunk > (p.gmerge ? kMaxChunksGlobal : kMaxCluster) || p.T > kMaxT || p.d != kD)
+    return cudaErrorInvalidValue;
   if (!tcmap::make_map(&mq, p.q, p.d, p.Hq, p.T, p.B, p.q_sh, p.q_st, p.q_sb, G, kRows / G) ||
       !tcmap::make_map(&mk, p.kc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, kKeys) ||
       !tcmap::make_map(&mv, p.vc, p.d, p.Hkv, p.Lmax, p.B, p.kv_sh, p.kv_sl, p.kv_sb, 1, kKeys))
@@ -775,7 +867,7 @@ cudaError_t launch_attn_pair(const AttnParams& p, cudaStream_t stream) {
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.gmerge ? 0 : 1;         // chunks merged through the workspace need no cluster
   e = cudaLaunchKernelEx(&cfg, attn_pair_kernel, mq, mk, mv, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -47,6 +47,7 @@ bool ws_ok(const void* ws, size_t ws_bytes, size_t need) {
 struct AttnPlan {
   bool tc;            // tensor-core prefix kernel
   bool pair;          // ... in its two-query-tile form (attn_pair.cu)
+  bool gmerge;        // ... with its chunks merged through the workspace
   bool sparse;
   bool tc_sparse;     // block top-k on the tensor-core kernel
   int nchunk, chunk_len, node_tile, nblk_max;
@@ -79,6 +80,12 @@ tv_status check_attn(const tv_attn_args* a) {
 // long-context and Llama-3-8B-shaped workloads.
 constexpr double kPairTile = 1.5;
 constexpr double kPairFixed = 6.0;
+// The two-tile CTA whose chunks merge through the workspace: no cluster (so
+// any number of chunks up to 16 and no co-scheduling of a pair's chunks),
+// for a fixed cost 1.5 tiles higher (its rows written out and, by the last
+// chunk, read back).
+constexpr double kPairGlobalFixed = 7.5;
+constexpr int kPairGlobalMaxChunks = 16;
 
 AttnPlan plan_attn(const tv_attn_args* a) {
   AttnPlan pl;
@@ -121,18 +128,23 @@ AttnPlan plan_attn(const tv_attn_args* a) {
       const bool pair_ok = a->T <= 2048;
       double best = 1e300;
       int64_t best_len = tiles;
-      for (int form = 0; form < (pair_ok ? 2 : 1); ++form) {
-        for (int c = 1; c <= 8; ++c) {
+      // forms: 0 one tile per CTA, 1 a tile pair (chunks in a cluster), 2 a
+      // tile pair with its chunks merged through the workspace (2..16
+      // chunks, as many CTAs as the device holds at once)
+      const bool global_ok = pair_ok && units_pair <= kMaxTickets;
+      for (int form = 0; form < (pair_ok ? (global_ok ? 3 : 2) : 1); ++form) {
+        for (int c = (form == 2 ? 2 : 1); c <= (form == 2 ? kPairGlobalMaxChunks : 8); ++c) {
           const int64_t lt = (tiles + c - 1) / c;
           if (c > 1 && lt < 4) break;                       // at least four tiles per chunk
           if ((tiles + lt - 1) / lt != c) continue;          // c chunks not realisable
-          const int act = form ? attn_pair_active_clusters(c) : attn_tc_active_clusters(c);
+          const int act = form == 2 ? attn_pair_active_clusters(1)
+                                    : (form ? attn_pair_active_clusters(c) : attn_tc_active_clusters(c));
           if (act <= 0) continue;
-          const int64_t u = form ? units_pair : units;
+          const int64_t u = form == 2 ? units_pair * c : (form ? units_pair : units);
           const double waves = static_cast<double>((u + act - 1) / act);
-          const double cost = waves * (form ? kPairFixed + static_cast<double>(lt) * kPairTile
-                                            : 3.0 + static_cast<double>(lt));
-          if (cost < best) { best = cost; best_len = lt; pl.pair = form == 1; }
+          const double fixed = form == 2 ? kPairGlobalFixed : (form ? kPairFixed : 3.0);
+          const double cost = waves * (fixed + static_cast<double>(lt) * (form ? kPairTile : 1.0));
+          if (cost < best) { best = cost; best_len = lt; pl.pair = form >= 1; pl.gmerge = form == 2; }
         }
       }
       len = best_len * 128;
@@ -146,8 +158,17 @@ AttnPlan plan_attn(const tv_attn_args* a) {
   // partials (prefix chunks + the tree-path partial) through the workspace
   const size_t nparts = (pl.tc || pl.tc_sparse) ? 0 : static_cast<size_t>(pl.nchunk) + 1;
   size_t off = kTicketBytes;
-  pl.off_o = off;  off = align256(off + nparts * rows * a->d * sizeof(float));
-  pl.off_lse = off; off = align256(off + nparts * rows * sizeof(float));
+  if (pl.gmerge) {
+    // the two-tile kernel's workspace merge: per (pair, chunk) both tiles'
+    // 128 rows of d fp32 values and their log-sum-exps
+    const int64_t ntiles2 = (a->T + pl.node_tile - 1) / pl.node_tile;
+    const size_t slots = static_cast<size_t>(a->B) * a->Hkv * ((ntiles2 + 1) / 2) * pl.nchunk * 2 * 128;
+    pl.off_o = off;  off = align256(off + slots * a->d * sizeof(float));
+    pl.off_lse = off; off = align256(off + slots * sizeof(float));
+  } else {
+    pl.off_o = off;  off = align256(off + nparts * rows * a->d * sizeof(float));
+    pl.off_lse = off; off = align256(off + nparts * rows * sizeof(float));
+  }
   pl.off_ok = off;  off = align256(off + static_cast<size_t>(a->B) * a->T * sizeof(int32_t));
   if (pl.sparse) {
     pl.nblk_max = (a->Lmax + a->block_size - 1) / a->block_size;
@@ -175,7 +196,7 @@ extern "C" size_t tree_verify_attn_workspace_size(const tv_attn_args* a) {
 extern "C" int32_t tv_attn_path(const tv_attn_args* a) {
   if (check_attn(a) != TV_OK) return -1;
   const AttnPlan pl = plan_attn(a);
-  return pl.sparse ? (pl.tc_sparse ? 3 : 2) : (pl.tc ? (pl.pair ? 4 : 1) : 0);
+  return pl.sparse ? (pl.tc_sparse ? 3 : 2) : (pl.tc ? (pl.pair ? (pl.gmerge ? 5 : 4) : 1) : 0);
 }
 
 extern "C" int32_t tv_attn_launches(const tv_attn_args* a) {
@@ -210,6 +231,7 @@ extern "C" tv_status tree_verify_attn(const tv_attn_args* a, void* ws, size_t ws
   p.lse = a->lse;
   p.status = a->dev_status;
   p.prefix_only = a->prefix_only;
+  p.gmerge = pl.gmerge ? 1 : 0;
   p.nchunk = pl.nchunk; p.chunk_len = pl.chunk_len; p.node_tile = pl.node_tile;
   unsigned char* w = static_cast<unsigned char*>(ws);
   p.part_o = reinterpret_cast<float*>(w + pl.off_o);

@@ -108,4 +108,4 @@ class Iteration:
         self.emitted += n + 1
 
     def launches_per_step(self):
-        return 1 + 2 * self.rounds + self.tv.last_attn_launches + 1 + 1
+        return 1 + self.rounds + self.tv.last_attn_launches + 1 + 1
