@@ -760,11 +760,12 @@ __device__ void row_body(const ExpandParams& p, int r, unsigned char* dsm, Expan
   };
   bool ok = true;
 
-  // one lane per warp waits for a staged chunk (the warp then reads it)
+  // every lane waits for a staged chunk itself (measured faster than one
+  // lane per warp followed by a warp barrier)
   const uint32_t lost = g_row_wait_polls;
   auto wait_chunk = [&](int c) {
     bool w = true;
-    if (lane == 0) {
+    if (lane == 0 || lost == 0u) {
       if (c == 0 && lost != 0u) {
         // the test hook: the first phase of a barrier nothing arrives on
         w = false;
@@ -774,8 +775,7 @@ __device__ void row_body(const ExpandParams& p, int r, unsigned char* dsm, Expan
         w = tc::mbar_wait(&sh.bar[c], 0, &sh.abort);
       }
     }
-    __syncwarp();
-    return __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
+    return __all_sync(0xffffffffu, w);
   };
 
   // the histogram frame: maximum and minimum of the first chunk
