@@ -11,21 +11,29 @@
 // their cursors.  (Tokens past the remaining budget can never be taken.)
 //
 // One launch per round, one CTA per row (expand_round_kernel):
-//   row      the row is staged in shared memory by bulk copies (when it
-//            fits); its maximum and minimum, then its lse (fp64) with a
-//            histogram of 2048 value bins over [min, max] (monotone in the
-//            logit, so bin order is rank order and the bin holding the K-th
-//            element follows from a prefix count); the elements of the bins
+//   row      the row is copied into shared memory at kernel entry (bulk
+//            copies in 16 KB chunks, when it fits).  The first chunk gives
+//            the frame of a 2048-bin value histogram (its maximum and
+//            minimum; values outside share the first or last bin, and bin
+//            order is rank order) and a collection threshold.  Pass 1, chunk
+//            by chunk as the copies land: finiteness, the row maximum, the
+//            histogram, and the collection of the elements at or above the
+//            threshold (about 1.5 K of them).  Pass 2: the row's lse in fp64
+//            (a table-driven exponential).  The bin of the K-th largest
+//            follows from one scan of the histogram; the collected elements
 //            above it are scattered bin by bin into the node's list and
 //            ordered inside their bin by counting, the boundary bin's best
 //            members likewise.  Crowded bins fall back to a bitonic sort of
-//            the whole list, a boundary bin too crowded for shared memory
-//            to a radix select on the 32-bit key.
+//            the whole list, a boundary bin too crowded for shared memory to
+//            a radix select on the 32-bit key, a collection that missed part
+//            of the top K to a scatter from the row.
 //   merge    the last CTA to finish its row (a ticket) takes the best
 //            s <= 128 candidates of the union, repeatedly: the s-th best
-//            list head bounds the s-th best candidate, so only entries at
-//            least as good as the worst head in the first s (found with a
-//            histogram of the heads' scores) can be taken; they are
+//            list head (heads are cached in the node metadata) bounds the
+//            s-th best candidate, so only entries at least as good as the
+//            worst head in the first s (found with a histogram of the
+//            heads' scores; with fewer than s heads, the s-th best of the
+//            first ceil(s / H) entries of every list) can be taken; they are
 //            gathered, a histogram of their scores isolates the s winners
 //            (exact (score, parent, token) ranks inside the boundary bin),
 //            the winners are ordered by counting and appended.  When a
