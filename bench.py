@@ -19,7 +19,7 @@ the 8 TB/s / 2.25 PFLOP/s denominators.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--config longctx|longctx_sparse|specexec70b|serving|llama3_8b|tiny]
-                    [--only] [--no-cpu-baseline] [--split-prefix]
+                    [--only] [--no-cpu-baseline] [--split-prefix | --iteration]
 
 --iteration replays one whole speculative iteration (tree expansion with a
 random-weight drafter stand-in, a random-weight target layer and
