@@ -967,33 +967,23 @@ def run_split_prefix(args, rank, world, dev, flush):
     partials are all-gathered over NCCL and merged by log-sum-exp with
     tree_verify_attn_merge.  A step = partial + all-gather + merge, timed
     with CUDA events (max over ranks); `value` counts each tree token once."""
-    import tree_verification_verify_b200 as tv
     from synth import config_attn_case
+    from tree_verification_verify_b200.split import prefix_slice, split_tree_verify_attn
     a = config_attn_case("longctx", seed=0, device=dev)
     B, T, Hq, d = a.q.shape
     Lmax = a.k_cache.shape[1]
-    lo, hi = (rank * Lmax) // world, ((rank + 1) * Lmax) // world
+    lo, hi = prefix_slice(rank, world, Lmax)
     L = a.prefix_len.cpu().numpy()
-    pl = torch.from_numpy(np.clip(L - lo, 0, hi - lo).astype(np.int32)).to(dev)
     kc, vc = a.k_cache[:, lo:hi], a.v_cache[:, lo:hi]
-    part_o = torch.empty_like(a.q)
-    part_l = torch.empty(B, T, Hq, dtype=torch.float32, device=dev)
-    all_o = torch.empty((world,) + tuple(a.q.shape), dtype=a.q.dtype, device=dev)
-    all_l = torch.empty(world, B, T, Hq, dtype=torch.float32, device=dev)
+    parts = (torch.empty_like(a.q), torch.empty(B, T, Hq, dtype=torch.float32, device=dev),
+             torch.empty((world,) + tuple(a.q.shape), dtype=a.q.dtype, device=dev),
+             torch.empty(world, B, T, Hq, dtype=torch.float32, device=dev))
     out = torch.empty_like(a.q)
-    lse = torch.empty_like(part_l)
+    lse = torch.empty(B, T, Hq, dtype=torch.float32, device=dev)
 
     def one():
-        tv.tree_verify_attn(a.q, kc, vc, pl, a.k_tree, a.v_tree, a.parent, out=part_o, lse=part_l,
-                            prefix_only=(rank != world - 1))
-        if world > 1:
-            import torch.distributed as dist
-            dist.all_gather_into_tensor(all_o, part_o)
-            dist.all_gather_into_tensor(all_l, part_l)
-        else:
-            all_o[0].copy_(part_o)
-            all_l[0].copy_(part_l)
-        tv.tree_verify_attn_merge(all_o, all_l, out=out, lse=lse)
+        split_tree_verify_attn(a.q, kc, vc, a.prefix_len, a.k_tree, a.v_tree, a.parent, rank, world, lo, hi,
+                               parts=parts, out=out, lse=lse)
 
     for _ in range(args.warmup):
         flush.zero_()

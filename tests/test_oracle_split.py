@@ -109,11 +109,10 @@ def _rank(rank, world, port, q):
     dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     T = 13
     case = attn_case(2, T, 8, 2, 32, [333, 120], "fp32", tree_bfs_fanout(T, (3, 2)), seed=7)
+    from tree_verification_verify_b200.split import prefix_slice, slice_prefix_len
     Lmax = case.k_cache.shape[1]
-    per = (Lmax + world - 1) // world
-    lo, hi = rank * per, min(Lmax, (rank + 1) * per)
-    L = case.prefix_len.numpy()
-    pl = torch.from_numpy(np.clip(L - lo, 0, hi - lo).astype(np.int32))
+    lo, hi = prefix_slice(rank, world, Lmax)       # the partition the GPU split uses
+    pl = slice_prefix_len(case.prefix_len, lo, hi)
     part = attn(case.q, case.k_cache[:, lo:hi], case.v_cache[:, lo:hi], pl, case.k_tree, case.v_tree, case.parent,
                 prefix_only=(rank != world - 1))
     o = torch.from_numpy(np.nan_to_num(part["out"], nan=0.0))
@@ -130,9 +129,10 @@ def _rank(rank, world, port, q):
 
 
 def test_two_ranks_gather_and_merge():
-    """Each of two gloo ranks attends to its half of the prefix (the last
-    rank with the tree keys), the partials are all-gathered, and every rank
-    merges them into the full tree attention."""
+    """Each of two gloo ranks attends to its slice of the prefix (the
+    partition of tree_verification_verify_b200.split; the last rank with the
+    tree keys), the partials are all-gathered, and every rank merges them
+    into the full tree attention."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -145,3 +145,20 @@ def test_two_ranks_gather_and_merge():
         assert p.exitcode == 0
     assert [r for r, _ in res] == [0, 1]
     assert all(e < 1e-12 for _, e in res), res
+
+
+def test_prefix_slices_partition_the_cache():
+    """The split's slices cover [0, Lmax) in rank order without overlap,
+    sizes within one row; each sequence's keys are counted once."""
+    from tree_verification_verify_b200.split import prefix_slice, slice_prefix_len
+    for Lmax in (0, 1, 7, 333, 131072):
+        for world in (1, 2, 3, 8):
+            sl = [prefix_slice(r, world, Lmax) for r in range(world)]
+            assert sl[0][0] == 0 and sl[-1][1] == Lmax
+            assert all(sl[r][1] == sl[r + 1][0] for r in range(world - 1))
+            sizes = [hi - lo for lo, hi in sl]
+            assert max(sizes) - min(sizes) <= 1
+            L = torch.tensor([0, min(1, Lmax), Lmax // 2, Lmax], dtype=torch.int32)
+            tot = sum(slice_prefix_len(L, lo, hi).to(torch.int64) for lo, hi in sl)
+            assert torch.equal(tot, L.to(torch.int64))
+
