@@ -1,7 +1,8 @@
 """Host-side logic of bench.py's JSON line, on CPU: the roofline denominators
 (measured peaks, else the stated fallback), the DRAM traffic taken from the
 committed ncu summary only while the kernel's source is the one captured,
-and the workload block of the line."""
+the workload block of the line, the attention's algorithmic FLOPs and bytes
+against a brute-force count, and the roofline fractions."""
 
 import hashlib
 import json
@@ -61,3 +62,55 @@ def test_config_block_names_the_workload():
     assert blk["parallelism"] == "replicas x2"
     assert "flush" in blk["l2"]
     assert "model" not in blk
+
+
+def _ancestor_counts(parent):
+    """|root path ∪ self| of every node, by walking parent[] (no helper of
+    the bench or of synth)."""
+    out = []
+    for i in range(len(parent)):
+        n, j = 0, i
+        while j >= 0:
+            n += 1
+            j = int(parent[j])
+        out.append(n)
+    return out
+
+
+def test_attention_work_counts_every_key_a_node_attends_to():
+    """attn_work's FLOPs and bytes against a brute-force count: node i of
+    sequence b attends to prefix_len[b] prefix keys plus its root path, two
+    matmuls of 2 d FLOPs per (query head, key); every prefix and tree K/V
+    element is read once."""
+    import numpy as np
+    rng = np.random.default_rng(3)
+    B, T, Hq, Hkv, d, elt = 3, 23, 8, 2, 64, 2
+    parents = []
+    for _ in range(B):
+        par = [-1] + [int(rng.integers(0, i)) for i in range(1, T)]
+        parents.append(par)
+    L = [0, 17, 1000]
+    flops, nbytes = bench.attn_work(parents, L, T, Hq, Hkv, d, elt)
+    keys = sum(L[b] + c for b in range(B) for c in _ancestor_counts(parents[b]))
+    assert flops == 4.0 * d * Hq * keys
+    assert nbytes == (sum(L) + B * T) * Hkv * d * 2 * elt
+    # block top-k: the kept prefix keys per (node, kv head) and the union of
+    # kept blocks replace the dense prefix
+    kept, union = 5 * 64 * B * T * Hkv, 9
+    f2, b2 = bench.attn_work(parents, L, T, Hq, Hkv, d, elt, kept_keys=kept, union_blocks=union,
+                             block_size=64, means_in_call=True)
+    path = sum(c for b in range(B) for c in _ancestor_counts(parents[b]))
+    assert f2 == 4.0 * d * (Hq // Hkv) * kept + 4.0 * d * Hq * path
+    assert b2 == union * 64 * d * 2 * elt + B * T * Hkv * d * 2 * elt + sum(L) * Hkv * d * elt
+
+
+def test_roofline_fractions_take_the_slower_bound(monkeypatch):
+    """The fraction is (the slower of bytes / bandwidth and FLOPs / peak) /
+    time, against both denominators."""
+    monkeypatch.setattr(bench, "peaks", lambda: (5000.0, 1000.0, "m", "m"))
+    r = bench.roofline_fracs(1e-3, nbytes=2.5e9, flops=0.0)          # 0.5 ms of HBM time
+    assert r["frac_measured"] == 0.5
+    assert r["frac_target"] == round(2.5e9 / 8000e9 / 1e-3, 4)
+    r = bench.roofline_fracs(2e-3, nbytes=1e9, flops=1e12)          # 1 ms of tensor time
+    assert r["frac_measured"] == 0.5
+    assert r["frac_target"] == round(1e12 / 2250e12 / 2e-3, 4)
