@@ -121,6 +121,18 @@ def roofline_fracs(seconds, nbytes=0.0, flops=0.0):
     return out
 
 
+def accept_work(parents, T, V, with_draft_probs):
+    """Algorithmic bytes of one tree_accept call: every node's target row
+    (V fp32 values) and, when draft probabilities are given, the draft row
+    of every node that has children (the rows its children were drawn
+    from)."""
+    internal = 0
+    if with_draft_probs:
+        for par in parents:
+            internal += len(set(int(x) for x in list(par)[1:T] if x >= 0))
+    return float(len(parents) * T * V * 4 + internal * V * 4)
+
+
 # --------------------------------------------------------------------------
 # distributed plumbing
 # --------------------------------------------------------------------------
@@ -326,11 +338,7 @@ class Step:
         else:
             self.attn_flops, self.attn_bytes = attn_work(par, L, T, Hq, Hkv, d, elt)
         V = self.acc.target_logits.shape[2]
-        internal = 0
-        if self.acc.draft_probs is not None:
-            for b in range(B):
-                internal += len(set(par[b][1:].tolist()))
-        self.accept_bytes = float(B * T * V * 4 + internal * V * 4)
+        self.accept_bytes = accept_work(par, T, V, self.acc.draft_probs is not None)
         self.expand_bytes = 0.0
         if self.expand:
             self.expand_bytes = float(sum(x.numel() for x in self.exp_logits) * 4)

@@ -114,3 +114,15 @@ def test_roofline_fractions_take_the_slower_bound(monkeypatch):
     r = bench.roofline_fracs(2e-3, nbytes=1e9, flops=1e12)          # 1 ms of tensor time
     assert r["frac_measured"] == 0.5
     assert r["frac_target"] == round(1e12 / 2250e12 / 2e-3, 4)
+
+
+def test_acceptance_bytes_read_the_rows_the_walk_needs():
+    """accept_work: B T target rows, plus one draft row per node with at
+    least one child when draft probabilities are given."""
+    import numpy as np
+    rng = np.random.default_rng(5)
+    B, T, V = 4, 19, 1000
+    parents = [np.array([-1] + [int(rng.integers(0, i)) for i in range(1, T)]) for _ in range(B)]
+    with_children = sum(sum(1 for j in range(T) if any(par[i] == j for i in range(1, T))) for par in parents)
+    assert bench.accept_work(parents, T, V, True) == (B * T + with_children) * V * 4
+    assert bench.accept_work(parents, T, V, False) == B * T * V * 4
