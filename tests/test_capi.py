@@ -113,3 +113,36 @@ def test_pool_bytes_grow_with_budget(L):
     assert 0 < a < b
     assert b >= 2048 * 2047 * 8
     assert L.tree_expand_pool_bytes(0, 10) == 0
+
+
+def test_host_argument_checks_of_the_split_beam_and_diagnostic_calls(L):
+    """The later entry points reject bad arguments on the host, before any
+    launch: the partial merge, prefix-only partials, the expansion mode and
+    the exponential diagnostic."""
+    import tree_verification_verify_b200 as tv
+    m = tv.AttnMergeArgs()
+    m.dtype, m.N, m.B, m.T, m.Hq, m.d = 1, 0, 1, 1, 1, 128           # N < 1
+    assert L.tree_verify_attn_merge(ctypes.byref(m), None) == 1
+    m.N = 65                                                        # more partials than supported
+    assert L.tree_verify_attn_merge(ctypes.byref(m), None) == 2
+    m.N, m.d = 2, 96                                                # d unsupported
+    assert L.tree_verify_attn_merge(ctypes.byref(m), None) == 2
+    m.d, m.dtype = 128, 7                                           # unknown dtype
+    assert L.tree_verify_attn_merge(ctypes.byref(m), None) == 1
+    m.dtype = 1                                                     # rows but no arrays
+    assert L.tree_verify_attn_merge(ctypes.byref(m), None) == 1
+    m.B = 0                                                         # nothing to merge
+    assert L.tree_verify_attn_merge(ctypes.byref(m), None) == 0
+    at = tv.AttnArgs()
+    at.dtype, at.B, at.T, at.Hq, at.Hkv, at.d = 1, 1, 1, 8, 2, 128
+    at.sparse_topk, at.block_size, at.prefix_only = 4, 64, 1        # prefix-only with block top-k
+    assert L.tree_verify_attn(ctypes.byref(at), None, 0, None) == 2
+    assert L.tv_attn_path(ctypes.byref(at)) == -1
+    at.sparse_topk, at.prefix_only = 0, 2                           # prefix_only is 0 or 1
+    assert L.tree_verify_attn(ctypes.byref(at), None, 0, None) == 1
+    e = tv.ExpandArgs()
+    e.V, e.R, e.Bsel, e.budget, e.draft_temperature, e.mode = 10, 0, 4, 16, 1.0, 5   # unknown mode
+    assert L.tree_expand_topb(ctypes.byref(e), None, 0, None) == 1
+    assert L.tv_expand_exp(None, None, -1, None) == 1               # n < 0
+    assert L.tv_expand_exp(None, None, 0, None) == 0                # nothing to do
+    assert L.tv_expand_exp(None, None, 3, None) == 1                # arrays missing
